@@ -1,0 +1,247 @@
+"""ctypes binding for libfa.so (argument marshalling only).
+
+Every function here checks the torch tensors it is given (device, dtype, shape,
+contiguity), passes raw device pointers and the current CUDA stream to the C
+ABI declared in include/fa.h, and raises FAError on a non-zero status.  No
+arithmetic of the attention itself happens in Python: if libfa.so is missing,
+loading fails loudly instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import pathlib
+
+import torch
+
+LIB_PATH = pathlib.Path(__file__).resolve().with_name("libfa.so")
+
+# Exported C symbols (the full list declared in include/fa.h).
+SYMBOLS = (
+    "fa_fwd", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess",
+    "fa_bwd_dkdv", "fa_bwd_dq", "fa_status_string", "fa_device_status", "fa_version",
+)
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def load_library() -> ctypes.CDLL:
+    """Loads libfa.so (built in-tree by exact_attention_107_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not LIB_PATH.exists():
+        raise RuntimeError(f"{LIB_PATH} is missing; build it with `python -m exact_attention_107_b200.build`")
+    lib = ctypes.CDLL(str(LIB_PATH))
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_fwd_f32.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_bwd_workspace_size.restype = sz
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
+    lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, i, i, i, i, vp]
+    lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_status_string.argtypes = [i]
+    lib.fa_status_string.restype = ctypes.c_char_p
+    lib.fa_device_status.argtypes = [i]
+    lib.fa_version.argtypes = []
+    for name in ("fa_fwd", "fa_fwd_f32", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq",
+                 "fa_device_status", "fa_version"):
+        getattr(lib, name).restype = i
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().fa_status_string(int(status)).decode()
+
+
+def _p(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _raise(st: int, where: str) -> None:
+    if st != 0:
+        raise FAError(st, where)
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)
+
+
+# ----------------------------------------------------------------------------- C-ABI calls
+def fa_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> None:
+    """O, lse <- attention(q, k, v); bf16 (B,H,N,D) tensors, lse (B,H,N) float32."""
+    B, H, N, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _check(t, name, torch.bfloat16, (B, H, N, D))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    _raise(load_library().fa_fwd(_p(q), _p(k), _p(v), _p(o), _p(lse), B, H, N, D, float(scale), int(causal),
+                                 _stream(stream)), "fa_fwd")
+
+
+def fa_fwd_f32(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> None:
+    """fp32 forward: float32 (B,H,N,D) tensors, lse (B,H,N) float32."""
+    B, H, N, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _check(t, name, torch.float32, (B, H, N, D))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    _raise(load_library().fa_fwd_f32(_p(q), _p(k), _p(v), _p(o), _p(lse), B, H, N, D, float(scale), int(causal),
+                                     _stream(stream)), "fa_fwd_f32")
+
+
+def fa_bwd_workspace_size(B: int, H: int, N: int, D: int) -> int:
+    return int(load_library().fa_bwd_workspace_size(B, H, N, D))
+
+
+def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, causal: bool, stream=None) -> None:
+    """dq, dk, dv <- gradients of attention; workspace: uint8 CUDA tensor of fa_bwd_workspace_size bytes."""
+    B, H, N, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _check(t, name, torch.bfloat16, (B, H, N, D))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    if not (workspace.is_cuda and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    nbytes = workspace.numel() * workspace.element_size()
+    _raise(load_library().fa_bwd(_p(q), _p(k), _p(v), _p(o), _p(do), _p(lse), _p(dq), _p(dk), _p(dv),
+                                 _p(workspace), nbytes, B, H, N, D, float(scale), int(causal), _stream(stream)),
+           "fa_bwd")
+
+
+def fa_bwd_preprocess(o, do, delta, stream=None) -> None:
+    B, H, N, D = o.shape
+    _check(o, "o", torch.bfloat16, (B, H, N, D))
+    _check(do, "do", torch.bfloat16, (B, H, N, D))
+    _check(delta, "delta", torch.float32, (B, H, N))
+    _raise(load_library().fa_bwd_preprocess(_p(o), _p(do), _p(delta), B, H, N, D, _stream(stream)),
+           "fa_bwd_preprocess")
+
+
+def fa_bwd_dkdv(q, k, v, do, lse, delta, dk, dv, scale: float, causal: bool, stream=None) -> None:
+    B, H, N, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("do", do), ("dk", dk), ("dv", dv)):
+        _check(t, name, torch.bfloat16, (B, H, N, D))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    _check(delta, "delta", torch.float32, (B, H, N))
+    _raise(load_library().fa_bwd_dkdv(_p(q), _p(k), _p(v), _p(do), _p(lse), _p(delta), _p(dk), _p(dv),
+                                      B, H, N, D, float(scale), int(causal), _stream(stream)), "fa_bwd_dkdv")
+
+
+def fa_bwd_dq(q, k, v, do, lse, delta, dq, scale: float, causal: bool, stream=None) -> None:
+    B, H, N, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("do", do), ("dq", dq)):
+        _check(t, name, torch.bfloat16, (B, H, N, D))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    _check(delta, "delta", torch.float32, (B, H, N))
+    _raise(load_library().fa_bwd_dq(_p(q), _p(k), _p(v), _p(do), _p(lse), _p(delta), _p(dq),
+                                    B, H, N, D, float(scale), int(causal), _stream(stream)), "fa_bwd_dq")
+
+
+def fa_device_status(reset: bool = False) -> int:
+    return int(load_library().fa_device_status(int(reset)))
+
+
+def fa_version() -> int:
+    return int(load_library().fa_version())
+
+
+# ----------------------------------------------------------------------------- convenience API
+def attention_forward(q, k, v, scale: float | None = None, causal: bool = False, stream=None):
+    """Returns (O, lse).  bf16 inputs use the tensor-core path, float32 inputs the fp32 path."""
+    B, H, N, D = q.shape
+    scale = default_scale(D) if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, N, device=q.device, dtype=torch.float32)
+    if q.dtype == torch.float32:
+        fa_fwd_f32(q, k, v, o, lse, scale, causal, stream)
+    else:
+        fa_fwd(q, k, v, o, lse, scale, causal, stream)
+    return o, lse
+
+
+def attention_backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, stream=None,
+                       workspace=None):
+    """Returns (dQ, dK, dV) for bf16 inputs."""
+    B, H, N, D = q.shape
+    scale = default_scale(D) if scale is None else scale
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if workspace is None:
+        workspace = torch.empty(fa_bwd_workspace_size(B, H, N, D), device=q.device, dtype=torch.uint8)
+    fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal, stream)
+    return dq, dk, dv
+
+
+class FlashAttention(torch.autograd.Function):
+    """autograd wrapper: forward saves (q, k, v, O, lse); backward recomputes P from lse."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, scale, causal):
+        o, lse = attention_forward(q, k, v, scale, causal)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.scale, ctx.causal = scale, causal
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = attention_backward(q, k, v, o, lse, do.contiguous(), ctx.scale, ctx.causal)
+        return dq, dk, dv, None, None
+
+
+def flash_attention(q, k, v, scale: float | None = None, causal: bool = False):
+    """Differentiable exact attention on bf16 (B,H,N,D) CUDA tensors."""
+    return FlashAttention.apply(q, k, v, default_scale(q.shape[-1]) if scale is None else scale, causal)
+
+
+def attention_fwd_bwd_from_host(q_h, k_h, v_h, do_h, scale: float, causal: bool, dev_bufs=None, out=None,
+                                stream=None):
+    """One full step from host memory: copy q, k, v, dO (pinned host tensors) to the
+    device, run forward and backward, and copy O, lse, dQ, dK, dV back to `out`
+    (pinned host tensors, allocated when None).  Returns (out, h2d_bytes, d2h_bytes)."""
+    B, H, N, D = q_h.shape
+    if dev_bufs is None:
+        dev = torch.device("cuda")
+        dev_bufs = {n: torch.empty(B, H, N, D, device=dev, dtype=torch.bfloat16)
+                    for n in ("q", "k", "v", "do", "o", "dq", "dk", "dv")}
+        dev_bufs["lse"] = torch.empty(B, H, N, device=dev, dtype=torch.float32)
+        dev_bufs["ws"] = torch.empty(fa_bwd_workspace_size(B, H, N, D), device=dev, dtype=torch.uint8)
+    if out is None:
+        out = {n: torch.empty(B, H, N, D, dtype=torch.bfloat16).pin_memory() for n in ("o", "dq", "dk", "dv")}
+        out["lse"] = torch.empty(B, H, N, dtype=torch.float32).pin_memory()
+    d = dev_bufs
+    for n, h in (("q", q_h), ("k", k_h), ("v", v_h), ("do", do_h)):
+        d[n].copy_(h, non_blocking=True)
+    fa_fwd(d["q"], d["k"], d["v"], d["o"], d["lse"], scale, causal, stream)
+    fa_bwd(d["q"], d["k"], d["v"], d["o"], d["do"], d["lse"], d["dq"], d["dk"], d["dv"], d["ws"], scale, causal,
+           stream)
+    for n in ("o", "lse", "dq", "dk", "dv"):
+        out[n].copy_(d[n], non_blocking=True)
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, do_h))
+    d2h = sum(t.numel() * t.element_size() for t in out.values())
+    return out, h2d, d2h

@@ -1,0 +1,262 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument validation, TMA tensor
+// maps, per-device state, and kernel launches.  No entry point allocates memory,
+// synchronises the host (except fa_device_status) or throws.
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_internal.h"
+
+namespace {
+
+// Device status word: kernels record the first device-side failure here
+// (FA_ERR_TIMEOUT when a pipeline wait exceeded its limit).
+__device__ int g_fa_status;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  bool sm100 = false;
+  int num_sms = 0;
+  int* status = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// Per-device set-up (once per device, with that device current): architecture,
+// SM count and the device address of the status word.
+int device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  DeviceState& s = g_dev[dev];
+  std::call_once(s.once, [&s, dev] {
+    int major = 0, minor = 0;
+    s.err = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (s.err == cudaSuccess) s.err = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (s.err == cudaSuccess) s.err = cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (s.err == cudaSuccess) s.err = cudaGetSymbolAddress(reinterpret_cast<void**>(&s.status), g_fa_status);
+    s.sm100 = (major == 10 && minor == 0);
+  });
+  if (s.err != cudaSuccess) return FA_ERR_CUDA;
+  if (!s.sm100) return FA_ERR_UNSUPPORTED_ARCH;
+  *out = &s;
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_shape(int B, int H, int N, int D, bool bf16) {
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
+  if (bf16 ? (D != 64 && D != 128) : (D != 32 && D != 64 && D != 128)) return FA_ERR_HEADDIM;
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh > INT_MAX / 2) return FA_ERR_SHAPE;
+  // Elements per tensor must stay addressable with 64-bit offsets and the TMA
+  // (dims < 2^32); grid size (ceil(N/256) * B*H) must fit a 31-bit grid.
+  if ((static_cast<long long>(N) + 255) / 256 * bh > INT_MAX) return FA_ERR_SHAPE;
+  return FA_OK;
+}
+
+// 3-D (D, N, B*H) bf16 tensor map, box 64 x box_rows x 1, 128-byte swizzle.
+int make_tmap(CUtensorMap* map, const void* ptr, int BH, int N, int D, int box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return FA_ERR_LAUNCH;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
+}
+
+int launch_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH; }
+
+bool scale_ok(float scale) { return std::isfinite(scale) && scale > 0.f; }
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 10000; }
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_NULL: return "FA_ERR_NULL: a required pointer is NULL";
+    case FA_ERR_SHAPE: return "FA_ERR_SHAPE: B, H or N out of range";
+    case FA_ERR_HEADDIM: return "FA_ERR_HEADDIM: unsupported head dimension";
+    case FA_ERR_ALIGN: return "FA_ERR_ALIGN: pointer not 16-byte aligned";
+    case FA_ERR_UNSUPPORTED_ARCH: return "FA_ERR_UNSUPPORTED_ARCH: device is not sm_100";
+    case FA_ERR_LAUNCH: return "FA_ERR_LAUNCH: kernel launch or tensor-map encoding failed";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a device-side wait exceeded its limit";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing or too small";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA runtime error";
+    case FA_ERR_ARG: return "FA_ERR_ARG: invalid argument";
+    default: return "unknown fa_status";
+  }
+}
+
+int fa_device_status(int reset) {
+  DeviceState* ds = nullptr;
+  int st = device_state(&ds);
+  if (st != FA_OK) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_fa_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (reset) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_fa_status, &zero, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return v;
+}
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int D,
+           float scale, int causal, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  int st = check_shape(B, H, N, D, true);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
+  if (!scale_ok(scale) || (causal != 0 && causal != 1)) return FA_ERR_ARG;
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  fa::FwdLaunch a{};
+  const int BH = B * H;
+  if ((st = make_tmap(&a.tmQ, q, BH, N, D, 128)) != FA_OK) return st;
+  if ((st = make_tmap(&a.tmK, k, BH, N, D, 128)) != FA_OK) return st;
+  if ((st = make_tmap(&a.tmV, v, BH, N, D, 128)) != FA_OK) return st;
+  if ((st = make_tmap(&a.tmO, o, BH, N, D, 32)) != FA_OK) return st;
+  a.lse = lse;
+  a.BH = BH;
+  a.N = N;
+  a.D = D;
+  a.scale = scale;
+  a.causal = causal;
+  a.status = ds->status;
+  a.num_sms = ds->num_sms;
+  return launch_status(fa::launch_fwd_bf16(a, static_cast<cudaStream_t>(stream)));
+}
+
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N, int D,
+               float scale, int causal, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
+  int st = check_shape(B, H, N, D, false);
+  if (st != FA_OK) return st;
+  if (static_cast<long long>(B) * H > 65535) return FA_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
+  if (!scale_ok(scale) || (causal != 0 && causal != 1)) return FA_ERR_ARG;
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  return launch_status(
+      fa::launch_fwd_f32(q, k, v, o, lse, B * H, N, D, scale, causal, static_cast<cudaStream_t>(stream)));
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int D) {
+  if (check_shape(B, H, N, D, true) != FA_OK) return 0;
+  const size_t bytes = static_cast<size_t>(B) * H * N * sizeof(float);
+  return (bytes + 255) / 256 * 256;
+}
+
+int fa_bwd_preprocess(const void* o, const void* dO, float* delta, int B, int H, int N, int D, void* stream) {
+  if (!o || !dO || !delta) return FA_ERR_NULL;
+  int st = check_shape(B, H, N, D, true);
+  if (st != FA_OK) return st;
+  if (!aligned16(o) || !aligned16(dO) || !aligned16(delta)) return FA_ERR_ALIGN;
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  return launch_status(fa::launch_bwd_preprocess(o, dO, delta, static_cast<long long>(B) * H * N, D,
+                                                 static_cast<cudaStream_t>(stream)));
+}
+
+static int bwd_common(const void* q, const void* k, const void* v, const void* dO, const float* lse,
+                      const float* delta, int B, int H, int N, int D, float scale, int causal,
+                      fa::BwdLaunch* a) {
+  if (!q || !k || !v || !dO || !lse || !delta) return FA_ERR_NULL;
+  int st = check_shape(B, H, N, D, true);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(lse) || !aligned16(delta))
+    return FA_ERR_ALIGN;
+  if (!scale_ok(scale) || (causal != 0 && causal != 1)) return FA_ERR_ARG;
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  const int BH = B * H;
+  if ((st = make_tmap(&a->tmQ, q, BH, N, D, 128)) != FA_OK) return st;
+  if ((st = make_tmap(&a->tmK, k, BH, N, D, 128)) != FA_OK) return st;
+  if ((st = make_tmap(&a->tmV, v, BH, N, D, 128)) != FA_OK) return st;
+  if ((st = make_tmap(&a->tmdO, dO, BH, N, D, 128)) != FA_OK) return st;
+  a->lse = lse;
+  a->delta = delta;
+  a->BH = BH;
+  a->N = N;
+  a->D = D;
+  a->scale = scale;
+  a->causal = causal;
+  a->status = ds->status;
+  a->num_sms = ds->num_sms;
+  return FA_OK;
+}
+
+int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, const float* lse, const float* delta,
+                void* dk, void* dv, int B, int H, int N, int D, float scale, int causal, void* stream) {
+  if (!dk || !dv) return FA_ERR_NULL;
+  if (!aligned16(dk) || !aligned16(dv)) return FA_ERR_ALIGN;
+  fa::BwdLaunch a{};
+  int st = bwd_common(q, k, v, dO, lse, delta, B, H, N, D, scale, causal, &a);
+  if (st != FA_OK) return st;
+  if ((st = make_tmap(&a.tmdK, dk, a.BH, N, D, 32)) != FA_OK) return st;
+  if ((st = make_tmap(&a.tmdV, dv, a.BH, N, D, 32)) != FA_OK) return st;
+  return launch_status(fa::launch_bwd_dkdv(a, static_cast<cudaStream_t>(stream)));
+}
+
+int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO, const float* lse, const float* delta,
+              void* dq, int B, int H, int N, int D, float scale, int causal, void* stream) {
+  if (!dq) return FA_ERR_NULL;
+  if (!aligned16(dq)) return FA_ERR_ALIGN;
+  fa::BwdLaunch a{};
+  int st = bwd_common(q, k, v, dO, lse, delta, B, H, N, D, scale, causal, &a);
+  if (st != FA_OK) return st;
+  if ((st = make_tmap(&a.tmdQ, dq, a.BH, N, D, 32)) != FA_OK) return st;
+  return launch_status(fa::launch_bwd_dq(a, static_cast<cudaStream_t>(stream)));
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
+           void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int D, float scale,
+           int causal, void* stream) {
+  if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_NULL;
+  int st = check_shape(B, H, N, D, true);
+  if (st != FA_OK) return st;
+  if (!workspace || workspace_bytes < fa_bwd_workspace_size(B, H, N, D)) return FA_ERR_WORKSPACE;
+  // Validate everything the three stages will check, so that an error launches nothing.
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return FA_ERR_ALIGN;
+  if (!scale_ok(scale) || (causal != 0 && causal != 1)) return FA_ERR_ARG;
+  float* delta = static_cast<float*>(workspace);
+  if ((st = fa_bwd_preprocess(o, dO, delta, B, H, N, D, stream)) != FA_OK) return st;
+  if ((st = fa_bwd_dkdv(q, k, v, dO, lse, delta, dk, dv, B, H, N, D, scale, causal, stream)) != FA_OK) return st;
+  return fa_bwd_dq(q, k, v, dO, lse, delta, dq, B, H, N, D, scale, causal, stream);
+}
+
+}  // extern "C"

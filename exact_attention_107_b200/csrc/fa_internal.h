@@ -1,0 +1,47 @@
+// fa_internal.h -- launch interfaces between the C ABI (fa_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+constexpr int kStatusTimeout = 7;  // FA_ERR_TIMEOUT
+
+// bf16 forward (fa_fwd_sm100.cu).  Tensor maps are 3-D (D, N, B*H) bf16 with
+// 64 x 128 x 1 boxes and 128-byte swizzle.
+struct FwdLaunch {
+  CUtensorMap tmQ, tmK, tmV, tmO;
+  float* lse;
+  int BH, N, D;
+  float scale;
+  int causal;
+  int* status;
+  int num_sms;
+};
+cudaError_t launch_fwd_bf16(const FwdLaunch& a, cudaStream_t stream);
+
+// fp32 forward (fa_fwd_f32.cu), plain pointers.
+cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
+                           int BH, int N, int D, float scale, int causal, cudaStream_t stream);
+
+// Backward stage 1 (fa_bwd_sm100.cu): delta = rowsum(dO * O).
+cudaError_t launch_bwd_preprocess(const void* o, const void* dO, float* delta, long long rows, int D,
+                                  cudaStream_t stream);
+
+// Backward stages 2 and 3 (fa_bwd_sm100.cu).
+struct BwdLaunch {
+  CUtensorMap tmQ, tmK, tmV, tmdO;   // loads
+  CUtensorMap tmdQ, tmdK, tmdV;      // stores
+  const float* lse;
+  const float* delta;
+  int BH, N, D;
+  float scale;
+  int causal;
+  int* status;
+  int num_sms;
+};
+cudaError_t launch_bwd_dkdv(const BwdLaunch& a, cudaStream_t stream);
+cudaError_t launch_bwd_dq(const BwdLaunch& a, cudaStream_t stream);
+
+}  // namespace fa

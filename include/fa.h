@@ -1,0 +1,124 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact, IO-aware tiled attention for NVIDIA B200 (sm_100a).
+ *
+ * The operation (all entry points):
+ *     S   = scale * Q K^T                (N x N per batch b and head h)
+ *     S_ij = -inf for j > i               (only when causal != 0; top-left aligned)
+ *     P   = softmax(S) row-wise,  O = P V
+ *     lse_i = ln( sum_j exp(S_ij) )       (natural-log logsumexp of the scaled scores)
+ * This is the attention of the three-line PyTorch form in "CUDA-kernel-level
+ * optimisation: why Flash Attention is 5-10x faster than native PyTorch"
+ * (guanweilu.cn, section "three lines of PyTorch"), computed the way its
+ * section "three tricks" and "LLM paper notes #8: FlashAttention" (adg.csdn.net,
+ * sections "tiling", "online softmax", "recomputation") describe: Q/K/V tiles
+ * staged on chip, an online softmax with a running max and sum, no N x N matrix
+ * in device memory, and a backward pass that recomputes P from lse.
+ *
+ * Conventions shared by every entry point
+ *   - Layout: every tensor is contiguous (B, H, N, D), head dimension innermost
+ *     (the layout of naive_attention in "Flash Attention principles: making
+ *     Transformers faster", ijyty.com, section "memory bottleneck").  lse and
+ *     delta are contiguous (B, H, N) float32.
+ *   - Pointers are DEVICE pointers (cudaMalloc'd or equivalent) on the current
+ *     device, 16-byte aligned.  The caller owns and allocates every buffer; the
+ *     library never allocates or frees device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Every call is asynchronous on that stream; the library does no
+ *     host synchronisation.
+ *   - Supported: B, H, N >= 1; D in {64, 128} for bf16; D in {32, 64, 128} for
+ *     fp32; Nq == Nk == N; causal in {0, 1}; B*H <= 65535*... (see fa_check).
+ *   - Return value: FA_OK (0) or an fa_status code.  Arguments are validated
+ *     before anything is launched; on an error nothing is launched and no
+ *     output is touched.  Errors are never thrown across the ABI.
+ *   - Device-side failures (a pipeline wait that exceeded its time limit) do
+ *     not trap: the kernel records FA_ERR_TIMEOUT in a device status word and
+ *     returns; fa_device_status() reads (and optionally clears) that word.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_NULL = 1,             /* a required pointer is NULL                      */
+  FA_ERR_SHAPE = 2,            /* B, H or N out of range, or index overflow       */
+  FA_ERR_HEADDIM = 3,          /* unsupported head dimension D                    */
+  FA_ERR_ALIGN = 4,            /* a pointer is not 16-byte aligned                */
+  FA_ERR_UNSUPPORTED_ARCH = 5, /* current device is not sm_100 (B200)             */
+  FA_ERR_LAUNCH = 6,           /* cudaLaunch / tensor-map encoding failed         */
+  FA_ERR_TIMEOUT = 7,          /* a device-side wait exceeded its limit           */
+  FA_ERR_WORKSPACE = 8,        /* workspace NULL or smaller than required         */
+  FA_ERR_CUDA = 9,             /* another CUDA runtime error                      */
+  FA_ERR_ARG = 10              /* another invalid argument (scale not finite ...) */
+} fa_status;
+
+/* Forward, bf16 in / bf16 out, fp32 accumulation (tcgen05 tensor cores).
+ *   q, k, v : (B,H,N,D) bf16, read only.
+ *   o       : (B,H,N,D) bf16, written (O = P V, rounded to nearest even).
+ *   lse     : (B,H,N) float32, written (natural-log logsumexp of scale*q.k).
+ *   scale   : the softmax scale (e.g. 1/sqrt(D)); must be finite and > 0.
+ *   causal  : 0 = full attention, 1 = key j allowed for query i iff j <= i. */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int H, int N, int D, float scale, int causal, void* stream);
+
+/* Forward in fp32 throughout (fp32 in, fp32 FFMA arithmetic, fp32 out), for
+ * callers that need ~1e-6 relative accuracy.  Same arguments as fa_fwd with
+ * float32 tensors. */
+int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
+               int B, int H, int N, int D, float scale, int causal, void* stream);
+
+/* Bytes of device workspace fa_bwd needs: the per-row term
+ * delta_i = sum_d dO_id * O_id as (B,H,N) float32, rounded up to 256 bytes. */
+size_t fa_bwd_workspace_size(int B, int H, int N, int D);
+
+/* Backward, bf16 (recomputes P from lse; never stores an N x N matrix).
+ *   q, k, v, o, dO : (B,H,N,D) bf16 inputs; o and lse must be the outputs of
+ *                    fa_fwd for the same q, k, v, scale and causal.
+ *   lse            : (B,H,N) float32 from fa_fwd.
+ *   dq, dk, dv     : (B,H,N,D) bf16, overwritten (not accumulated into).
+ *   workspace      : device buffer of at least fa_bwd_workspace_size() bytes,
+ *                    contents on entry ignored, clobbered on exit.
+ * Equivalent to fa_bwd_preprocess, then fa_bwd_dkdv and fa_bwd_dq on the
+ * same stream. */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
+           const float* lse, void* dq, void* dk, void* dv,
+           void* workspace, size_t workspace_bytes,
+           int B, int H, int N, int D, float scale, int causal, void* stream);
+
+/* Backward stage 1: delta (B,H,N) float32 = rowsum(dO * O) (fp32 arithmetic). */
+int fa_bwd_preprocess(const void* o, const void* dO, float* delta,
+                      int B, int H, int N, int D, void* stream);
+
+/* Backward stage 2: dK, dV (bf16, overwritten).  Each key tile is owned by one
+ * CTA that walks the query tiles, so dK and dV need no atomics. */
+int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
+                const float* lse, const float* delta, void* dk, void* dv,
+                int B, int H, int N, int D, float scale, int causal, void* stream);
+
+/* Backward stage 3: dQ (bf16, overwritten).  Each query tile is owned by one
+ * CTA that walks the key tiles, so dQ needs no atomics. */
+int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
+              const float* lse, const float* delta, void* dq,
+              int B, int H, int N, int D, float scale, int causal, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fa_status_string(int status);
+
+/* Reads the device status word of the current device (synchronises the
+ * device first).  Returns FA_OK or the first FA_ERR_* a kernel recorded;
+ * if reset != 0 the word is cleared afterwards. */
+int fa_device_status(int reset);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

@@ -1,0 +1,58 @@
+"""Helpers for comparing the CUDA path with the fp64 oracle (tests only).
+
+Tolerances (bf16 inputs, fp32 accumulation), applied in fp64 on the CPU:
+    O       relative Frobenius <= 5e-3 and max-abs <= 2e-2
+    lse     max-abs <= 1e-3
+    dQ/dK/dV relative Frobenius <= 1e-2 each
+fp32 path: O relative Frobenius <= 1e-5, lse max-abs <= 1e-5 * max(1, |lse|).
+"""
+from __future__ import annotations
+
+import torch
+
+import exact_attention_107_b200 as fa
+
+TOL = {"O_fro": 5e-3, "O_max": 2e-2, "lse_max": 1e-3, "grad_fro": 1e-2, "f32_fro": 1e-5, "f32_lse": 1e-5}
+
+
+def rel_fro(a, b) -> float:
+    a, b = a.double(), b.double()
+    return ((a - b).norm() / b.norm().clamp_min(1e-300)).item()
+
+
+def max_abs(a, b) -> float:
+    return (a.double() - b.double()).abs().max().item()
+
+
+def check_fwd(O, lse, ref_O, ref_lse, label=""):
+    e = {"O_fro": rel_fro(O, ref_O), "O_max": max_abs(O, ref_O), "lse_max": max_abs(lse, ref_lse)}
+    assert e["O_fro"] <= TOL["O_fro"], (label, e)
+    assert e["O_max"] <= TOL["O_max"], (label, e)
+    assert e["lse_max"] <= TOL["lse_max"], (label, e)
+    return e
+
+
+def check_grads(got: dict, ref: dict, label=""):
+    e = {n: rel_fro(got[n], ref[n]) for n in ("dQ", "dK", "dV")}
+    for n, v in e.items():
+        assert v <= TOL["grad_fro"], (label, n, e)
+    return e
+
+
+def gpu_forward(q, k, v, scale, causal):
+    dev = torch.device("cuda")
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    O, lse = fa.attention_forward(qd, kd, vd, scale, causal)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status(reset=True) == 0
+    return O, lse, (qd, kd, vd)
+
+
+def gpu_fwd_bwd(q, k, v, do, scale, causal):
+    dev = torch.device("cuda")
+    O, lse, (qd, kd, vd) = gpu_forward(q, k, v, scale, causal)
+    dod = do.to(dev)
+    dq, dk, dv = fa.attention_backward(qd, kd, vd, O, lse, dod, scale, causal)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status(reset=True) == 0
+    return {"O": O.cpu(), "lse": lse.cpu(), "dQ": dq.cpu(), "dK": dk.cpu(), "dV": dv.cpu()}

@@ -1,0 +1,91 @@
+"""Boundary tests that need no GPU: libfa.so loads, exports every symbol that
+include/fa.h declares, and rejects bad arguments with the documented status
+codes before touching any device."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+import exact_attention_107_b200 as fa
+
+HEADER = Path(__file__).resolve().parents[1] / "include" / "fa.h"
+
+
+def declared_functions():
+    text = HEADER.read_text()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(fa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert declared_functions() == sorted(fa.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = fa.load_library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings():
+    for code in range(11):
+        assert fa.status_string(code).startswith("FA_")
+    assert fa.status_string(999) == "unknown fa_status"
+
+
+def test_workspace_size():
+    assert fa.fa_bwd_workspace_size(1, 8, 65536, 128) == 8 * 65536 * 4
+    assert fa.fa_bwd_workspace_size(1, 1, 3, 64) == 256          # rounded up to 256 bytes
+    assert fa.fa_bwd_workspace_size(1, 1, 128, 96) == 0          # unsupported D
+
+
+# Validation happens before any device call, so these run without a GPU.
+P = ctypes.c_void_p(0x10000)        # an aligned, never-dereferenced fake address
+U = ctypes.c_void_p(0x10008)        # misaligned
+Z = None
+
+
+def _fwd(q=P, k=P, v=P, o=P, lse=P, B=1, H=2, N=256, D=64, scale=0.125, causal=0):
+    return fa.load_library().fa_fwd(q, k, v, o, lse, B, H, N, D, scale, causal, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=Z), 1), (dict(lse=Z), 1),
+    (dict(B=0), 2), (dict(N=0), 2), (dict(H=-1), 2), (dict(B=2**30, H=2**30), 2),
+    (dict(D=96), 3), (dict(D=32), 3), (dict(D=256), 3),
+    (dict(k=U), 4), (dict(o=U), 4),
+    (dict(scale=float("nan")), 10), (dict(scale=0.0), 10), (dict(scale=-1.0), 10), (dict(causal=2), 10),
+])
+def test_fwd_rejects_bad_arguments(kw, code):
+    assert _fwd(**kw) == code
+
+
+def test_fwd_f32_rejects_bad_arguments():
+    lib = fa.load_library()
+    assert lib.fa_fwd_f32(Z, P, P, P, P, 1, 1, 64, 64, 0.1, 0, None) == 1
+    assert lib.fa_fwd_f32(P, P, P, P, P, 1, 1, 64, 48, 0.1, 0, None) == 3
+    assert lib.fa_fwd_f32(P, P, P, P, P, 300, 300, 64, 64, 0.1, 0, None) == 2   # B*H > 65535
+
+
+def test_bwd_rejects_bad_arguments():
+    lib = fa.load_library()
+    ws = lib.fa_bwd_workspace_size(1, 2, 256, 64)
+    args = [P] * 9
+    assert lib.fa_bwd(*args, P, ws, 1, 2, 256, 64, 0.125, 0, None) != 6       # reaches the device check
+    assert lib.fa_bwd(*args, Z, ws, 1, 2, 256, 64, 0.125, 0, None) == 8       # no workspace
+    assert lib.fa_bwd(*args, P, ws - 1, 1, 2, 256, 64, 0.125, 0, None) == 8   # too small
+    assert lib.fa_bwd(*args[:8], U, P, ws, 1, 2, 256, 64, 0.125, 0, None) == 4
+    assert lib.fa_bwd(*args[:3], Z, *args[4:], P, ws, 1, 2, 256, 64, 0.125, 0, None) == 1
+    assert lib.fa_bwd(*args, P, ws, 1, 2, 256, 80, 0.125, 0, None) == 3
+    assert lib.fa_bwd_dq(P, P, P, P, P, P, Z, 1, 1, 128, 64, 0.1, 0, None) == 1
+    assert lib.fa_bwd_dkdv(P, P, P, P, P, P, P, U, 1, 1, 128, 64, 0.1, 0, None) == 4
+    assert lib.fa_bwd_preprocess(P, P, Z, 1, 1, 128, 64, None) == 1
+
+
+def test_binding_requires_cuda_tensors():
+    import torch
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.fa_fwd(q, q, q, q, torch.zeros(1, 1, 128), 0.125, False)
