@@ -17,6 +17,7 @@ from ._binding import (  # noqa: F401
     fa_bwd,
     fa_bwd_dkdv,
     fa_bwd_dq,
+    fa_bwd_noalloc,
     fa_bwd_preprocess,
     fa_bwd_workspace_size,
     fa_device_status,

@@ -20,6 +20,7 @@ LIB_PATH = pathlib.Path(__file__).resolve().with_name("libfa.so")
 SYMBOLS = (
     "fa_fwd", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess",
     "fa_bwd_dkdv", "fa_bwd_dq", "fa_status_string", "fa_device_status", "fa_version",
+    "fa_bwd_noalloc",
 )
 
 _lib = None
@@ -48,6 +49,8 @@ def load_library() -> ctypes.CDLL:
     lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, i, i, i, i, vp]
     lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_bwd_noalloc.restype = i
     lib.fa_status_string.argtypes = [i]
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_device_status.argtypes = [i]
@@ -132,6 +135,20 @@ def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, causal: boo
     _raise(load_library().fa_bwd(_p(q), _p(k), _p(v), _p(o), _p(do), _p(lse), _p(dq), _p(dk), _p(dv),
                                  _p(workspace), nbytes, B, H, N, D, float(scale), int(causal), _stream(stream)),
            "fa_bwd")
+
+
+def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, stream=None) -> None:
+    """Like fa_bwd but with no workspace: for callers that cannot allocate device
+    memory (they are handed only input and output buffers).  Uses the library's
+    fixed scratch array, so problems with B*H*N > 2,097,152 rows are rejected and
+    calls that overlap on the GPU must not share it."""
+    B, H, N, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _check(t, name, torch.bfloat16, (B, H, N, D))
+    _check(lse, "lse", torch.float32, (B, H, N))
+    _raise(load_library().fa_bwd_noalloc(_p(q), _p(k), _p(v), _p(o), _p(do), _p(lse), _p(dq), _p(dk), _p(dv),
+                                         B, H, N, D, float(scale), int(causal), _stream(stream)),
+           "fa_bwd_noalloc")
 
 
 def fa_bwd_preprocess(o, do, delta, stream=None) -> None:

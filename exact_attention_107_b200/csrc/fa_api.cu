@@ -115,6 +115,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing or too small";
     case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA runtime error";
     case FA_ERR_ARG: return "FA_ERR_ARG: invalid argument";
+    case FA_ERR_NOALLOC_CAPACITY: return "FA_ERR_NOALLOC_CAPACITY: problem exceeds the fa_bwd_noalloc scratch size";
     default: return "unknown fa_status";
   }
 }

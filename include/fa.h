@@ -54,7 +54,8 @@ typedef enum {
   FA_ERR_TIMEOUT = 7,          /* a device-side wait exceeded its limit           */
   FA_ERR_WORKSPACE = 8,        /* workspace NULL or smaller than required         */
   FA_ERR_CUDA = 9,             /* another CUDA runtime error                      */
-  FA_ERR_ARG = 10              /* another invalid argument (scale not finite ...) */
+  FA_ERR_ARG = 10,             /* another invalid argument (scale not finite ...) */
+  FA_ERR_NOALLOC_CAPACITY = 11 /* problem too large for fa_bwd_noalloc's scratch   */
 } fa_status;
 
 /* Forward, bf16 in / bf16 out, fp32 accumulation (tcgen05 tensor cores).
@@ -105,6 +106,29 @@ int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
 int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
               const float* lse, const float* delta, void* dq,
               int B, int H, int N, int D, float scale, int causal, void* stream);
+
+/* Size of the fixed device scratch array that fa_bwd_noalloc uses (8 MiB). */
+#define FA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+/* Backward that allocates nothing and takes no workspace.  The paper has no
+ * counterpart to this entry point; it exists for callers that cannot allocate
+ * device memory -- code that a host framework hands only its input and output
+ * buffers, with all device memory planned up front and no workspace or allocator
+ * available to the operator.
+ *   Same arguments, layout, results and errors as fa_bwd, minus the workspace.
+ *   Scratch: a fixed FA_NOALLOC_SCRATCH_BYTES array in the library's own device
+ *     memory (held by every GPU that loads the library until the process exits).
+ *     Limit: fa_bwd_workspace_size(B, H, N, D) <= FA_NOALLOC_SCRATCH_BYTES,
+ *     i.e. B*H*N <= 2,097,152 rows; larger problems return
+ *     FA_ERR_NOALLOC_CAPACITY before anything is launched.
+ *   Set-up: the first call on a device looks up the array's device address
+ *     (with that device current); make that first call before any stream capture.
+ *   Sharing: every call uses the same array; nothing in it needs to start at zero
+ *     (each call rewrites what it reads), but calls whose work overlaps on the GPU
+ *     (unordered streams) race on it. */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                   const float* lse, void* dq, void* dk, void* dv,
+                   int B, int H, int N, int D, float scale, int causal, void* stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(int status);
