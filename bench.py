@@ -165,7 +165,7 @@ def run_ours(args, rank, world, local_rank):
     o = torch.empty_like(q)
     lse = torch.empty(B, H, N, device=dev, dtype=torch.float32)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    delta = torch.empty(B, H, N, device=dev, dtype=torch.float32)
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, D), device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream(dev)
 
     names = ("fwd", "bwd_pre", "bwd_dkdv", "bwd_dq")
@@ -176,13 +176,13 @@ def run_ours(args, rank, world, local_rank):
         fa.fa_fwd(q, k, v, o, lse, scale, causal, stream)
         if ev is not None:
             ev[1].record(stream)
-        fa.fa_bwd_preprocess(o, do, delta, stream)
+        fa.fa_bwd_preprocess(o, do, lse, ws, stream)
         if ev is not None:
             ev[2].record(stream)
-        fa.fa_bwd_dkdv(q, k, v, do, lse, delta, dk, dv, scale, causal, stream)
+        fa.fa_bwd_dkdv(q, k, v, do, ws, dk, dv, scale, causal, stream)
         if ev is not None:
             ev[3].record(stream)
-        fa.fa_bwd_dq(q, k, v, do, lse, delta, dq, scale, causal, stream)
+        fa.fa_bwd_dq(q, k, v, do, ws, dq, scale, causal, stream)
         if ev is not None:
             ev[4].record(stream)
 
@@ -222,7 +222,7 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_e2e:
         pinned = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
         dev_bufs = {"q": q, "k": k, "v": v, "do": do, "o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv,
-                    "ws": torch.empty(fa.fa_bwd_workspace_size(B, H, N, D), device=dev, dtype=torch.uint8)}
+                    "ws": ws}
         out = {n: torch.empty(B, H, N, D, dtype=torch.bfloat16).pin_memory() for n in ("o", "dq", "dk", "dv")}
         out["lse"] = torch.empty(B, H, N, dtype=torch.float32).pin_memory()
         for _ in range(max(1, args.warmup)):

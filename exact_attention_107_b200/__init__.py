@@ -27,6 +27,7 @@ from ._binding import (  # noqa: F401
     flash_attention,
     load_library,
     status_string,
+    workspace_views,
 )
 
 __version__ = "1.0.0"

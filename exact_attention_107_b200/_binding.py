@@ -46,9 +46,9 @@ def load_library() -> ctypes.CDLL:
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.fa_bwd_workspace_size.restype = sz
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
-    lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, i, i, i, i, vp]
-    lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
-    lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, vp, sz, i, i, i, i, vp]
+    lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, sz, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, sz, vp, i, i, i, i, f, i, vp]
     lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_bwd_noalloc.restype = i
     lib.fa_status_string.argtypes = [i]
@@ -140,8 +140,8 @@ def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, causal: boo
 def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, stream=None) -> None:
     """Like fa_bwd but with no workspace: for callers that cannot allocate device
     memory (they are handed only input and output buffers).  Uses the library's
-    fixed scratch array, so problems with B*H*N > 2,097,152 rows are rejected and
-    calls that overlap on the GPU must not share it."""
+    fixed 8 MiB scratch array, so problems with B*H*ceil(N/128)*128 > 1,048,576
+    rows are rejected and calls that overlap on the GPU must not share it."""
     B, H, N, D = q.shape
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv)):
         _check(t, name, torch.bfloat16, (B, H, N, D))
@@ -151,33 +151,48 @@ def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, 
            "fa_bwd_noalloc")
 
 
-def fa_bwd_preprocess(o, do, delta, stream=None) -> None:
+def _ws(workspace):
+    if not (isinstance(workspace, torch.Tensor) and workspace.is_cuda and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return _p(workspace), workspace.numel() * workspace.element_size()
+
+
+def fa_bwd_preprocess(o, do, lse, workspace, stream=None) -> None:
+    """Backward stage 1: fills the workspace with -lse*log2(e) and delta = rowsum(dO * O)."""
     B, H, N, D = o.shape
     _check(o, "o", torch.bfloat16, (B, H, N, D))
     _check(do, "do", torch.bfloat16, (B, H, N, D))
-    _check(delta, "delta", torch.float32, (B, H, N))
-    _raise(load_library().fa_bwd_preprocess(_p(o), _p(do), _p(delta), B, H, N, D, _stream(stream)),
+    _check(lse, "lse", torch.float32, (B, H, N))
+    wp, wn = _ws(workspace)
+    _raise(load_library().fa_bwd_preprocess(_p(o), _p(do), _p(lse), wp, wn, B, H, N, D, _stream(stream)),
            "fa_bwd_preprocess")
 
 
-def fa_bwd_dkdv(q, k, v, do, lse, delta, dk, dv, scale: float, causal: bool, stream=None) -> None:
+def fa_bwd_dkdv(q, k, v, do, workspace, dk, dv, scale: float, causal: bool, stream=None) -> None:
+    """Backward stage 2: dK, dV from the workspace filled by fa_bwd_preprocess."""
     B, H, N, D = q.shape
     for name, t in (("q", q), ("k", k), ("v", v), ("do", do), ("dk", dk), ("dv", dv)):
         _check(t, name, torch.bfloat16, (B, H, N, D))
-    _check(lse, "lse", torch.float32, (B, H, N))
-    _check(delta, "delta", torch.float32, (B, H, N))
-    _raise(load_library().fa_bwd_dkdv(_p(q), _p(k), _p(v), _p(do), _p(lse), _p(delta), _p(dk), _p(dv),
+    wp, wn = _ws(workspace)
+    _raise(load_library().fa_bwd_dkdv(_p(q), _p(k), _p(v), _p(do), wp, wn, _p(dk), _p(dv),
                                       B, H, N, D, float(scale), int(causal), _stream(stream)), "fa_bwd_dkdv")
 
 
-def fa_bwd_dq(q, k, v, do, lse, delta, dq, scale: float, causal: bool, stream=None) -> None:
+def fa_bwd_dq(q, k, v, do, workspace, dq, scale: float, causal: bool, stream=None) -> None:
+    """Backward stage 3: dQ from the workspace filled by fa_bwd_preprocess."""
     B, H, N, D = q.shape
     for name, t in (("q", q), ("k", k), ("v", v), ("do", do), ("dq", dq)):
         _check(t, name, torch.bfloat16, (B, H, N, D))
-    _check(lse, "lse", torch.float32, (B, H, N))
-    _check(delta, "delta", torch.float32, (B, H, N))
-    _raise(load_library().fa_bwd_dq(_p(q), _p(k), _p(v), _p(do), _p(lse), _p(delta), _p(dq),
+    wp, wn = _ws(workspace)
+    _raise(load_library().fa_bwd_dq(_p(q), _p(k), _p(v), _p(do), wp, wn, _p(dq),
                                     B, H, N, D, float(scale), int(causal), _stream(stream)), "fa_bwd_dq")
+
+
+def workspace_views(workspace, B: int, H: int, N: int):
+    """(nl, delta) float32 views of a backward workspace, each (B, H, Npad)."""
+    npad = (N + 127) // 128 * 128
+    f = workspace.view(torch.float32)[: 2 * B * H * npad].view(2, B, H, npad)
+    return f[0], f[1]
 
 
 def fa_device_status(reset: bool = False) -> int:

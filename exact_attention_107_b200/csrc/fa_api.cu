@@ -72,9 +72,8 @@ int check_shape(int B, int H, int N, int D, bool bf16) {
   if (bf16 ? (D != 64 && D != 128) : (D != 32 && D != 64 && D != 128)) return FA_ERR_HEADDIM;
   const long long bh = static_cast<long long>(B) * H;
   if (bh > INT_MAX / 2) return FA_ERR_SHAPE;
-  // Elements per tensor must stay addressable with 64-bit offsets and the TMA
-  // (dims < 2^32); grid size (ceil(N/256) * B*H) must fit a 31-bit grid.
-  if ((static_cast<long long>(N) + 255) / 256 * bh > INT_MAX) return FA_ERR_SHAPE;
+  // The largest grid (ceil(N/128) * B*H CTAs, the dK/dV kernel) must fit a 31-bit grid.
+  if ((static_cast<long long>(N) + 127) / 128 * bh > INT_MAX) return FA_ERR_SHAPE;
   return FA_OK;
 }
 
@@ -176,39 +175,55 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int D) {
   if (check_shape(B, H, N, D, true) != FA_OK) return 0;
-  const size_t bytes = static_cast<size_t>(B) * H * N * sizeof(float);
-  return (bytes + 255) / 256 * 256;
+  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  return 2 * static_cast<size_t>(B) * H * npad * sizeof(float);    // a multiple of 1024 bytes
 }
 
-int fa_bwd_preprocess(const void* o, const void* dO, float* delta, int B, int H, int N, int D, void* stream) {
-  if (!o || !dO || !delta) return FA_ERR_NULL;
+// Workspace views: ws_nl = [0, B*H*Npad) floats, ws_delta = [B*H*Npad, 2*B*H*Npad).
+static int workspace_views(void* ws, size_t ws_bytes, int B, int H, int N, int D, fa::BwdLaunch* a) {
+  if (!ws || ws_bytes < fa_bwd_workspace_size(B, H, N, D)) return FA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return FA_ERR_ALIGN;
+  a->Npad = (N + 127) / 128 * 128;
+  a->ws_nl = static_cast<float*>(ws);
+  a->ws_delta = a->ws_nl + static_cast<size_t>(B) * H * a->Npad;
+  return FA_OK;
+}
+
+int fa_bwd_preprocess(const void* o, const void* dO, const float* lse, void* workspace, size_t workspace_bytes,
+                      int B, int H, int N, int D, void* stream) {
+  if (!o || !dO || !lse) return FA_ERR_NULL;
   int st = check_shape(B, H, N, D, true);
   if (st != FA_OK) return st;
-  if (!aligned16(o) || !aligned16(dO) || !aligned16(delta)) return FA_ERR_ALIGN;
+  if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return FA_ERR_ALIGN;
+  fa::BwdLaunch a{};
+  if ((st = workspace_views(workspace, workspace_bytes, B, H, N, D, &a)) != FA_OK) return st;
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
-  return launch_status(fa::launch_bwd_preprocess(o, dO, delta, static_cast<long long>(B) * H * N, D,
-                                                 static_cast<cudaStream_t>(stream)));
+  a.o = o;
+  a.dO = dO;
+  a.lse = lse;
+  a.BH = B * H;
+  a.N = N;
+  a.D = D;
+  return launch_status(fa::launch_bwd_preprocess(a, static_cast<cudaStream_t>(stream)));
 }
 
-static int bwd_common(const void* q, const void* k, const void* v, const void* dO, const float* lse,
-                      const float* delta, int B, int H, int N, int D, float scale, int causal,
+static int bwd_common(const void* q, const void* k, const void* v, const void* dO, const void* workspace,
+                      size_t workspace_bytes, int B, int H, int N, int D, float scale, int causal, int q_box_rows,
                       fa::BwdLaunch* a) {
-  if (!q || !k || !v || !dO || !lse || !delta) return FA_ERR_NULL;
+  if (!q || !k || !v || !dO) return FA_ERR_NULL;
   int st = check_shape(B, H, N, D, true);
   if (st != FA_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(lse) || !aligned16(delta))
-    return FA_ERR_ALIGN;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO)) return FA_ERR_ALIGN;
+  if ((st = workspace_views(const_cast<void*>(workspace), workspace_bytes, B, H, N, D, a)) != FA_OK) return st;
   if (!scale_ok(scale) || (causal != 0 && causal != 1)) return FA_ERR_ARG;
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
   const int BH = B * H;
-  if ((st = make_tmap(&a->tmQ, q, BH, N, D, 128)) != FA_OK) return st;
+  if ((st = make_tmap(&a->tmQ, q, BH, N, D, q_box_rows)) != FA_OK) return st;
   if ((st = make_tmap(&a->tmK, k, BH, N, D, 128)) != FA_OK) return st;
   if ((st = make_tmap(&a->tmV, v, BH, N, D, 128)) != FA_OK) return st;
-  if ((st = make_tmap(&a->tmdO, dO, BH, N, D, 128)) != FA_OK) return st;
-  a->lse = lse;
-  a->delta = delta;
+  if ((st = make_tmap(&a->tmdO, dO, BH, N, D, q_box_rows)) != FA_OK) return st;
   a->BH = BH;
   a->N = N;
   a->D = D;
@@ -219,24 +234,25 @@ static int bwd_common(const void* q, const void* k, const void* v, const void* d
   return FA_OK;
 }
 
-int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, const float* lse, const float* delta,
-                void* dk, void* dv, int B, int H, int N, int D, float scale, int causal, void* stream) {
+int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, const void* workspace,
+                size_t workspace_bytes, void* dk, void* dv, int B, int H, int N, int D, float scale, int causal,
+                void* stream) {
   if (!dk || !dv) return FA_ERR_NULL;
   if (!aligned16(dk) || !aligned16(dv)) return FA_ERR_ALIGN;
   fa::BwdLaunch a{};
-  int st = bwd_common(q, k, v, dO, lse, delta, B, H, N, D, scale, causal, &a);
+  int st = bwd_common(q, k, v, dO, workspace, workspace_bytes, B, H, N, D, scale, causal, 128, &a);
   if (st != FA_OK) return st;
   if ((st = make_tmap(&a.tmdK, dk, a.BH, N, D, 32)) != FA_OK) return st;
   if ((st = make_tmap(&a.tmdV, dv, a.BH, N, D, 32)) != FA_OK) return st;
   return launch_status(fa::launch_bwd_dkdv(a, static_cast<cudaStream_t>(stream)));
 }
 
-int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO, const float* lse, const float* delta,
-              void* dq, int B, int H, int N, int D, float scale, int causal, void* stream) {
+int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO, const void* workspace,
+              size_t workspace_bytes, void* dq, int B, int H, int N, int D, float scale, int causal, void* stream) {
   if (!dq) return FA_ERR_NULL;
   if (!aligned16(dq)) return FA_ERR_ALIGN;
   fa::BwdLaunch a{};
-  int st = bwd_common(q, k, v, dO, lse, delta, B, H, N, D, scale, causal, &a);
+  int st = bwd_common(q, k, v, dO, workspace, workspace_bytes, B, H, N, D, scale, causal, 128, &a);
   if (st != FA_OK) return st;
   if ((st = make_tmap(&a.tmdQ, dq, a.BH, N, D, 32)) != FA_OK) return st;
   return launch_status(fa::launch_bwd_dq(a, static_cast<cudaStream_t>(stream)));
@@ -254,10 +270,11 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
     return FA_ERR_ALIGN;
   if (!scale_ok(scale) || (causal != 0 && causal != 1)) return FA_ERR_ARG;
-  float* delta = static_cast<float*>(workspace);
-  if ((st = fa_bwd_preprocess(o, dO, delta, B, H, N, D, stream)) != FA_OK) return st;
-  if ((st = fa_bwd_dkdv(q, k, v, dO, lse, delta, dk, dv, B, H, N, D, scale, causal, stream)) != FA_OK) return st;
-  return fa_bwd_dq(q, k, v, dO, lse, delta, dq, B, H, N, D, scale, causal, stream);
+  if ((st = fa_bwd_preprocess(o, dO, lse, workspace, workspace_bytes, B, H, N, D, stream)) != FA_OK) return st;
+  if ((st = fa_bwd_dkdv(q, k, v, dO, workspace, workspace_bytes, dk, dv, B, H, N, D, scale, causal, stream)) !=
+      FA_OK)
+    return st;
+  return fa_bwd_dq(q, k, v, dO, workspace, workspace_bytes, dq, B, H, N, D, scale, causal, stream);
 }
 
 }  // extern "C"

@@ -9,18 +9,20 @@
 //     dS = P * (dP - delta),   dQ = scale * dS K,   dK = scale * dS^T Q.
 //
 // Three stages, all on the caller's stream:
-//   1. preprocess   delta = rowsum(dO * O) in fp32 (bandwidth bound)
-//   2. dkdv kernel  one CTA per 128-key tile j walks the query tiles i:
-//                     S^T = K_j Q_i^T, dP^T = V_j dO_i^T           (tensor memory)
-//                     P^T, dS^T computed by 128 threads, one key row each
-//                     dV_j += P^T dO_i, dK_j += dS^T Q_i             (A from tensor memory)
-//   3. dq kernel    one CTA per 128-query tile i walks the key tiles j:
-//                     S = Q_i K_j^T, dP = dO_i V_j^T, dS, dQ_i += dS K_j
-// Every output tile is owned by exactly one CTA, so there are no atomics, no
-// fp32 dQ accumulator in device memory and the result is deterministic; the
-// price is recomputing S and dP a second time in stage 3.
-//
-// The probabilities used for dS are the bf16-rounded P that also feeds dV.
+//   1. preprocess   per row: delta = rowsum(dO * O) and nl = -lse * log2(e), both fp32,
+//                   into a workspace padded per head to a multiple of 128 rows
+//                   (padding rows: nl = -inf so their P is 0, delta = 0)
+//   2. dkdv kernel  one CTA per 128-key tile walks the query tiles (128 rows):
+//                     S^T = K_j Q_i^T, dP^T = V_j dO_i^T      (M=128 keys, N=128 queries)
+//                     P^T, dS^T computed by 256 threads (a key row, half the queries each)
+//                     dV_j += P^T dO_i, dK_j += dS^T Q_i        (A operand read from TMEM)
+//                   S^T of the next query tile is computed while dS^T of this one is.
+//   3. dq kernel    one CTA per 256 queries (two 128-row tiles) walks the key tiles:
+//                     S = Q_i K_j^T, P, dP = dO_i V_j^T (written over S once S is
+//                     read), dS, dQ_i += dS K_j
+// Every output tile is owned by exactly one CTA: no atomics, no fp32 dQ accumulator
+// in device memory, deterministic results; the price is recomputing S and dP in
+// stage 3.  The probabilities used for dS are the bf16-rounded P that also feed dV.
 #include <cstdint>
 #include <math_constants.h>
 
@@ -30,21 +32,26 @@
 namespace fa {
 namespace {
 
-constexpr int kTileRows = 128;
-constexpr int kThreads = 256;           // warp 0 loads, warp 1 issues MMAs, warps 4-7 compute
+constexpr int kThreads = 384;   // warp 0 loads, warp 1 issues MMAs, warps 4-11 compute
 constexpr float kLog2e = 1.44269504088896340736f;
 
 // ----------------------------------------------------------------------------- stage 1
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
                                                              const __nv_bfloat16* __restrict__ dO,
-                                                             float* __restrict__ delta, long long rows) {
+                                                             const float* __restrict__ lse,
+                                                             float* __restrict__ ws_nl, float* __restrict__ ws_delta,
+                                                             int N, int Npad, long long padded_rows) {
   constexpr int kLanesPerRow = D / 8;   // each lane reads 8 bf16 (16 bytes) of O and of dO
   const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const long long row = gt / kLanesPerRow;
+  const long long prow = gt / kLanesPerRow;          // row in the padded (B*H, Npad) layout
   const int part = static_cast<int>(gt % kLanesPerRow);
+  const long long bh = prow / Npad;
+  const int n = static_cast<int>(prow % Npad);
+  const bool real = prow < padded_rows && n < N;
+  const long long row = bh * N + n;                  // row in the caller's (B*H, N) layout
   float acc = 0.f;
-  if (row < rows) {
+  if (real) {
     const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
     const uint4 b = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
     const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
@@ -56,15 +63,20 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16
   }
 #pragma unroll
   for (int off = kLanesPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (row < rows && part == 0) delta[row] = acc;
+  if (prow < padded_rows && part == 0) {
+    ws_delta[prow] = acc;
+    ws_nl[prow] = real ? -lse[row] * kLog2e : -CUDART_INF_F;
+  }
 }
 
 // ----------------------------------------------------------------------------- shared helpers
-template <int D>
-struct Tiles {
-  static constexpr int kBox = kTileRows * 64 * 2;   // 16 KB: 128 rows x 64 bf16, 128-byte swizzle
+// A tile of `rows` rows x D bf16 in shared memory, stored as D/64 boxes of rows x 128 bytes
+// in the TMA 128-byte-swizzled layout.
+template <int D, int ROWS>
+struct Tile {
+  static constexpr int kBox = ROWS * 128;
   static constexpr int kNBox = D / 64;
-  static constexpr int kTile = kBox * kNBox;
+  static constexpr int kBytes = kBox * kNBox;
 };
 
 // Copies this thread's accumulator row (D fp32 columns of tensor memory, times `mul`)
@@ -86,20 +98,21 @@ __device__ __forceinline__ void stage_row_bf16(uint32_t tacc, float mul, uint8_t
       v.y = pack_bf16(__uint_as_float(o[8 * q4 + 2]) * mul, __uint_as_float(o[8 * q4 + 3]) * mul);
       v.z = pack_bf16(__uint_as_float(o[8 * q4 + 4]) * mul, __uint_as_float(o[8 * q4 + 5]) * mul);
       v.w = pack_bf16(__uint_as_float(o[8 * q4 + 6]) * mul, __uint_as_float(o[8 * q4 + 7]) * mul);
-      *reinterpret_cast<uint4*>(stage + box * Tiles<D>::kBox + r * 128 + ((chunk ^ (r & 7)) << 4)) = v;
+      *reinterpret_cast<uint4*>(stage + box * Tile<D, 128>::kBox + r * 128 + ((chunk ^ (r & 7)) << 4)) = v;
     }
   }
 }
 
-// One warp stores its 32 staged rows with the TMA (tensor map box: 64 x 32 x 1).
+// One warp stores its 32 staged rows with the TMA (tensor map box: 64 x 32 x 1);
+// rows at or past n_rows are skipped (or clipped by the hardware).
 template <int D>
 __device__ __forceinline__ void store_warp_rows(const CUtensorMap* tm, uint32_t stage_s, int wrow, int row0, int bh,
                                                 int lane, int n_rows) {
   fence_async_smem();
   __syncwarp();
   if (lane == 0 && row0 + wrow < n_rows) {
-    for (int c = 0; c < Tiles<D>::kNBox; ++c)
-      tma_store_3d(tm, stage_s + c * Tiles<D>::kBox + wrow * 128, c * 64, row0 + wrow, bh);
+    for (int c = 0; c < Tile<D, 128>::kNBox; ++c)
+      tma_store_3d(tm, stage_s + c * Tile<D, 128>::kBox + wrow * 128, c * 64, row0 + wrow, bh);
     bulk_commit();
     bulk_wait_read0();
   }
@@ -109,21 +122,41 @@ __device__ __forceinline__ void store_warp_rows(const CUtensorMap* tm, uint32_t 
 __device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
+// K-major operand slice for K-step kk (16 bf16 = 32 bytes) of a swizzled tile with box size `box`.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk, int box) {
+  return sdesc_sw128(tile + (kk >> 2) * box + (kk & 3) * 32, 16, 1024);
+}
+// MN-major operand slice for K-step kk (16 rows of 128 bytes) of a swizzled tile whose
+// 64-column boxes are `box` bytes apart.
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk, int box) {
+  return sdesc_sw128(tile + kk * 2048, box, 1024);
+}
+
 // ----------------------------------------------------------------------------- stage 2: dK, dV
+// One CTA per 128-key tile walks the query tiles (128 rows each).  Every MMA is
+// M=128 x N=128 (or N=D): S^T and dP^T (shared-memory operands), dV and dK (A from
+// tensor memory).  Two warpgroups split the 128 query columns of S^T / dP^T (64
+// each); each writes its bf16 P^T / dS^T only into columns it has already read
+// (warpgroup 0: the first 32 of its range, warpgroup 1: the last 32), and the
+// K-step addresses of the dV / dK MMAs stitch the two halves back together.
+// Q and dO have separate 2-stage rings, each released right after its last use.
 template <int D>
 struct DkdvSmem {
-  using T = Tiles<D>;
-  static constexpr int kStages = 2;
-  static constexpr int kOffK = 0;                          // K_j (later dK staging)
-  static constexpr int kOffV = kOffK + T::kTile;           // V_j (later dV staging)
-  static constexpr int kOffQ = kOffV + T::kTile;           // [stage] Q_i
-  static constexpr int kOffdO = kOffQ + kStages * T::kTile;  // [stage] dO_i
-  static constexpr int kOffStat = kOffdO + kStages * T::kTile;  // [stage] -lse*log2e[128], delta[128]
-  static constexpr int kOffBar = kOffStat + kStages * 2 * kTileRows * 4;
+  using T = Tile<D, 128>;
+  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr int kOffK = 0;                                 // K_j (later dK staging)
+  static constexpr int kOffV = kOffK + T::kBytes;                 // V_j (later dV staging)
+  static constexpr int kOffQ = kOffV + T::kBytes;                 // [stage] Q_i
+  static constexpr int kOffdO = kOffQ + kStages * T::kBytes;      // [stage] dO_i
+  static constexpr int kOffStat = kOffdO + kStages * T::kBytes;   // [stage] nl[128], delta[128]
+  static constexpr int kStatBytes = 2 * 128 * 4;
+  static constexpr int kOffBar = kOffStat + kStages * kStatBytes;
   static constexpr int kBarKV = 0;
   static constexpr int kBarQFull = 1;
   static constexpr int kBarQEmpty = kBarQFull + kStages;
-  static constexpr int kBarS = kBarQEmpty + kStages;
+  static constexpr int kBarOFull = kBarQEmpty + kStages;
+  static constexpr int kBarOEmpty = kBarOFull + kStages;
+  static constexpr int kBarS = kBarOEmpty + kStages;
   static constexpr int kBarDP = kBarS + 1;
   static constexpr int kBarP = kBarDP + 1;
   static constexpr int kBarDS = kBarP + 1;
@@ -135,15 +168,22 @@ struct DkdvSmem {
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
+// Tensor-memory column of the packed bf16 pair for K-step kk (16 queries) of the
+// P^T (base 0) or dS^T (base 128) operand: queries 0-63 at base + [0, 32),
+// queries 64-127 at base + [96, 128).
+__device__ __forceinline__ uint32_t packed_col(uint32_t base, int kk) {
+  return base + (kk < 4 ? kk * 8 : 96 + (kk - 4) * 8);
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                     const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                    const float* __restrict__ lse, const float* __restrict__ delta, int N, int BH, int nt,
-                    float scale, int* status) {
+                    const float* __restrict__ ws_nl, const float* __restrict__ ws_delta, int N, int Npad, int BH,
+                    int nkt, float scale, int* status) {
   using L = DkdvSmem<D>;
-  using T = Tiles<D>;
+  using T = Tile<D, 128>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -152,30 +192,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Work item: key tile kt of head bh.  Causal: it meets query tiles kt..nt-1, so low
-  // kt are the heaviest and go first.
+  // Work item: key tile kt of head bh.  Causal: it meets query tiles kt..nkt-1, so
+  // low kt are the heaviest and go first.
   int kt, bh;
   if (CAUSAL) {
     kt = static_cast<int>(blockIdx.x / BH);
     bh = blockIdx.x % BH;
   } else {
-    kt = blockIdx.x % nt;
-    bh = blockIdx.x / nt;
+    kt = blockIdx.x % nkt;
+    bh = blockIdx.x / nkt;
   }
-  const int kv0 = kt * kTileRows;
+  const int kv0 = kt * 128;
   const int it0 = CAUSAL ? kt : 0;        // first query tile
-  const int n = nt - it0;                 // query tiles visited
+  const int n = nkt - it0;                // query tiles visited
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::kBarKV), 1);
     for (int s = 0; s < L::kStages; ++s) {
-      mbar_init(bar(L::kBarQFull + s), 2);   // TMA bytes + the warp's statistics
+      mbar_init(bar(L::kBarQFull + s), 1);
       mbar_init(bar(L::kBarQEmpty + s), 1);
+      mbar_init(bar(L::kBarOFull + s), 1);
+      mbar_init(bar(L::kBarOEmpty + s), 1);
     }
     mbar_init(bar(L::kBarS), 1);
     mbar_init(bar(L::kBarDP), 1);
-    mbar_init(bar(L::kBarP), kTileRows);
-    mbar_init(bar(L::kBarDS), kTileRows);
+    mbar_init(bar(L::kBarP), 256);
+    mbar_init(bar(L::kBarDS), 256);
     mbar_init(bar(L::kBarAcc), 1);
     mbar_init(bar(L::kBarMmaDone), 1);
     *abort_flag = 0;
@@ -189,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
-  // Tensor memory: S^T / P^T [0,128), dP^T / dS^T [128,256), dV [256,256+D), dK [256+D,256+2D)
+  // Tensor memory: S^T / P^T [0,128), dP^T / dS^T [128,256), dV [256,256+D), dK [256+D,256+2D).
   constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 256 + D;
 
   if (warp == 0) {
@@ -199,99 +241,99 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       prefetch_tmap(&tmdO);
-      mbar_arrive_expect_tx(bar(L::kBarKV), 2 * T::kTile);
+      mbar_arrive_expect_tx(bar(L::kBarKV), 2 * T::kBytes);
       for (int c = 0; c < T::kNBox; ++c) {
         tma_load_3d(sb + L::kOffK + c * T::kBox, &tmK, bar(L::kBarKV), c * 64, kv0, bh);
         tma_load_3d(sb + L::kOffV + c * T::kBox, &tmV, bar(L::kBarKV), c * 64, kv0, bh);
       }
-    }
-    int issued = 0;
-    bool ok = true;
-    for (int i = 0; i < n; ++i) {
-      const int s = i % L::kStages;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarQEmpty + s), ((i / L::kStages) & 1) ^ 1, abort_flag));
-      if (!ok) break;
-      const int q0 = (it0 + i) * kTileRows;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar(L::kBarQFull + s), 2 * T::kTile);
-        for (int c = 0; c < T::kNBox; ++c) {
-          tma_load_3d(sb + L::kOffQ + s * T::kTile + c * T::kBox, &tmQ, bar(L::kBarQFull + s), c * 64, q0, bh);
-          tma_load_3d(sb + L::kOffdO + s * T::kTile + c * T::kBox, &tmdO, bar(L::kBarQFull + s), c * 64, q0, bh);
-        }
+      int nq = 0, no = 0;
+      bool ok = true;
+      // Q_i (with the tile's row statistics) and dO_i, interleaved; each waits for its own ring.
+      for (int i = 0; i < n; ++i) {
+        const int s = i % L::kStages;
+        const uint32_t ph = ((i / L::kStages) & 1) ^ 1;
+        const int q0 = (it0 + i) * 128;
+        if (!(ok = mbar_wait(bar(L::kBarQEmpty + s), ph, abort_flag))) break;
+        const uint32_t qf = bar(L::kBarQFull + s);
+        mbar_arrive_expect_tx(qf, T::kBytes + L::kStatBytes);
+        for (int c = 0; c < T::kNBox; ++c)
+          tma_load_3d(sb + L::kOffQ + s * T::kBytes + c * T::kBox, &tmQ, qf, c * 64, q0, bh);
+        const size_t srow = static_cast<size_t>(bh) * Npad + q0;      // padded rows: always in bounds
+        bulk_load(sb + L::kOffStat + s * L::kStatBytes, ws_nl + srow, 128 * 4, qf);
+        bulk_load(sb + L::kOffStat + s * L::kStatBytes + 128 * 4, ws_delta + srow, 128 * 4, qf);
+        ++nq;
+        if (!(ok = mbar_wait(bar(L::kBarOEmpty + s), ph, abort_flag))) break;
+        const uint32_t of = bar(L::kBarOFull + s);
+        mbar_arrive_expect_tx(of, T::kBytes);
+        for (int c = 0; c < T::kNBox; ++c)
+          tma_load_3d(sb + L::kOffdO + s * T::kBytes + c * T::kBox, &tmdO, of, c * 64, q0, bh);
+        ++no;
       }
-      // Row statistics of this query tile; rows past N get P = 0 (lse = +inf) and delta = 0.
-      float* st = reinterpret_cast<float*>(smem + L::kOffStat + s * 2 * kTileRows * 4);
-      for (int c = lane; c < kTileRows; c += 32) {
-        const int qrow = q0 + c;
-        const bool in = qrow < N;
-        st[c] = in ? -lse[static_cast<size_t>(bh) * N + qrow] * kLog2e : -CUDART_INF_F;
-        st[kTileRows + c] = in ? delta[static_cast<size_t>(bh) * N + qrow] : 0.f;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::kBarQFull + s));
-      ++issued;
-    }
-    if (lane == 0) {
       if (!ok) raise_error(status, abort_flag, kStatusTimeout);
       mbar_wait_drain(bar(L::kBarKV), 0);
-      for (int i = max(0, issued - L::kStages); i < issued; ++i)
+      for (int i = max(0, nq - L::kStages); i < nq; ++i)
         mbar_wait_drain(bar(L::kBarQFull + i % L::kStages), (i / L::kStages) & 1);
+      for (int i = max(0, no - L::kStages); i < no; ++i)
+        mbar_wait_drain(bar(L::kBarOFull + i % L::kStages), (i / L::kStages) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(kTileRows, kTileRows, false, false);
-      constexpr uint32_t kIdAcc = idesc_bf16(kTileRows, D, false, true);
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // S^T, dP^T: K-major A and B
+      constexpr uint32_t kIdAcc = idesc_bf16(128, D, false, true);    // dV, dK: A in TMEM, B MN-major
       const uint32_t sK = sb + L::kOffK, sV = sb + L::kOffV;
-      // S^T = K_j Q_i^T and dP^T = V_j dO_i^T (both operands K-major)
-      auto issue_st = [&](int i) {
-        const uint32_t sQ = sb + L::kOffQ + (i % L::kStages) * T::kTile;
+      auto issue_st = [&](int i) {      // S^T = K_j Q_i^T
+        const uint32_t sQ = sb + L::kOffQ + (i % L::kStages) * T::kBytes;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * T::kBox + (kk & 3) * 32;
-          mma_ss(tmem + kColS, sdesc_sw128(sK + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024), kIdS, kk > 0);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + kColS, kmajor_desc(sK, kk, T::kBox), kmajor_desc(sQ, kk, T::kBox), kIdS, kk > 0);
         tc_commit(bar(L::kBarS));
       };
-      auto issue_dpt = [&](int i) {
-        const uint32_t sdO = sb + L::kOffdO + (i % L::kStages) * T::kTile;
+      auto issue_dpt = [&](int i) {     // dP^T = V_j dO_i^T
+        const uint32_t sdO = sb + L::kOffdO + (i % L::kStages) * T::kBytes;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * T::kBox + (kk & 3) * 32;
-          mma_ss(tmem + kColDP, sdesc_sw128(sV + off, 16, 1024), sdesc_sw128(sdO + off, 16, 1024), kIdS, kk > 0);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + kColDP, kmajor_desc(sV, kk, T::kBox), kmajor_desc(sdO, kk, T::kBox), kIdS, kk > 0);
         tc_commit(bar(L::kBarDP));
       };
-      // acc (+)= A_tmem [128 x 128 queries] * B_smem (queries x D, MN-major)
-      auto issue_acc = [&](uint32_t dcol, uint32_t acol, uint32_t b_tile, int i) {
+      // acc (+)= A_tmem (packed bf16, 128 queries) * B_smem (128 queries x D, MN-major)
+      auto issue_acc = [&](uint32_t dcol, uint32_t abase, uint32_t b_tile, bool first) {
 #pragma unroll
-        for (int kk = 0; kk < kTileRows / 16; ++kk)
-          mma_ts(tmem + dcol, tmem + acol + kk * 8, sdesc_sw128(b_tile + kk * 2048, T::kBox, 1024), kIdAcc,
-                 (i > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + dcol, tmem + packed_col(abase, kk), mnmajor_desc(b_tile, kk, T::kBox), kIdAcc,
+                 (!first || kk > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait(bar(L::kBarKV), 0, abort_flag);
-      for (int i = 0; ok && i < n; ++i) {
-        const int s = i % L::kStages;
-        if (i == 0) {
-          if (!(ok = mbar_wait(bar(L::kBarQFull), 0, abort_flag))) break;
+      if (ok && n > 0) {
+        ok = mbar_wait(bar(L::kBarQFull), 0, abort_flag) && mbar_wait(bar(L::kBarOFull), 0, abort_flag);
+        if (ok) {
           tc_fence_after();
           issue_st(0);
           issue_dpt(0);
         }
+      }
+      for (int i = 0; ok && i < n; ++i) {
+        const int s = i % L::kStages;
         if (!(ok = mbar_wait(bar(L::kBarP), i & 1, abort_flag))) break;
         tc_fence_after();
-        issue_acc(kColDV, kColS, sb + L::kOffdO + s * T::kTile, i);          // dV += P^T dO_i
+        issue_acc(kColDV, kColS, sb + L::kOffdO + s * T::kBytes, i == 0);        // dV += P^T dO_i
+        tc_commit(bar(L::kBarOEmpty + s));
         if (i + 1 < n) {
           const int sn = (i + 1) % L::kStages;
           if (!(ok = mbar_wait(bar(L::kBarQFull + sn), ((i + 1) / L::kStages) & 1, abort_flag))) break;
           tc_fence_after();
-          issue_st(i + 1);
+          issue_st(i + 1);                                                       // over P^T_i (read above)
         }
         if (!(ok = mbar_wait(bar(L::kBarDS), i & 1, abort_flag))) break;
         tc_fence_after();
-        issue_acc(kColDK, kColDP, sb + L::kOffQ + s * T::kTile, i);          // dK += dS^T Q_i
+        issue_acc(kColDK, kColDP, sb + L::kOffQ + s * T::kBytes, i == 0);        // dK += dS^T Q_i
         tc_commit(bar(L::kBarQEmpty + s));
-        if (i + 1 < n) issue_dpt(i + 1);
+        if (i + 1 < n) {
+          const int sn = (i + 1) % L::kStages;
+          if (!(ok = mbar_wait(bar(L::kBarOFull + sn), ((i + 1) / L::kStages) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_dpt(i + 1);                                                      // over dS^T_i (read above)
+        }
       }
       if (!ok) raise_error(status, abort_flag, kStatusTimeout);
       tc_commit(bar(L::kBarAcc));
@@ -300,49 +342,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ------------------------------------------------------------------ P^T, dS^T, epilogue
-    const int r = threadIdx.x - 128;                                    // key row = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tb = tmem + lane_off;
+    // ------------------------------------------------------------------ P^T, dS^T (64 query columns), epilogue
+    const int g = (warp - 4) >> 2;                                      // query columns [64g, 64g+64)
+    const int r = threadIdx.x - 128 * (1 + g);                           // key row = TMEM lane
+    const uint32_t tb = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t out_off = g == 0 ? 0 : 96;                            // where the packed half goes
     const int key = kv0 + r;
     const float scale_log2 = scale * kLog2e;
     bool ok = true;
     for (int i = 0; i < n; ++i) {
       const int s = i % L::kStages;
-      const int q0 = (it0 + i) * kTileRows;
-      const float* st = reinterpret_cast<const float*>(smem + L::kOffStat + s * 2 * kTileRows * 4);
+      const int q0 = (it0 + i) * 128;
+      const float* st = reinterpret_cast<const float*>(smem + L::kOffStat + s * L::kStatBytes) + 64 * g;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarQFull + s), (i / L::kStages) & 1, abort_flag));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS), i & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[4][32];
-      tmem_ld32(tb + kColS, sr[0]);
-      tmem_ld32(tb + kColS + 32, sr[1]);
-      tmem_ld32(tb + kColS + 64, sr[2]);
-      tmem_ld32(tb + kColS + 96, sr[3]);
+      uint32_t sr[2][32];
+      tmem_ld32(tb + kColS + 64 * g, sr[0]);
+      tmem_ld32(tb + kColS + 64 * g + 32, sr[1]);
       tmem_ld_wait();
       reg_fence(sr[0]);
       reg_fence(sr[1]);
-      reg_fence(sr[2]);
-      reg_fence(sr[3]);
-      // P^T[r][c] = exp2(s * scale * log2e - lse_c * log2e); causal: zero where key > query
-      const bool diag = CAUSAL && (q0 < kv0 + kTileRows);
-      uint32_t pk[2][32];
+      // P^T[r][c] = exp2(s * scale * log2e + nl_c); causal: zero where key > query
+      const int qc0 = q0 + 64 * g;                                       // query of this thread's column 0
+      const bool diag = CAUSAL && (qc0 < key + 64);                      // some column may be masked
+      uint32_t pk[32];
 #pragma unroll
-      for (int c2 = 0; c2 < kTileRows / 2; ++c2) {
+      for (int c2 = 0; c2 < 32; ++c2) {
         const int c = 2 * c2;
-        const float4 nl = *reinterpret_cast<const float4*>(st + (c & ~3));
-        const float nl0 = (c & 2) ? nl.z : nl.x, nl1 = (c & 2) ? nl.w : nl.y;
-        float p0 = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), scale_log2, nl0));
-        float p1 = ex2_approx(fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), scale_log2, nl1));
+        const float2 nl = *reinterpret_cast<const float2*>(st + c);
+        float p0 = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), scale_log2, nl.x));
+        float p1 = ex2_approx(fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), scale_log2, nl.y));
         if (diag) {
-          if (key > q0 + c) p0 = 0.f;
-          if (key > q0 + c + 1) p1 = 0.f;
+          if (key > qc0 + c) p0 = 0.f;
+          if (key > qc0 + c + 1) p1 = 0.f;
         }
-        pk[c2 >> 5][c2 & 31] = pack_bf16(p0, p1);
+        pk[c2] = pack_bf16(p0, p1);
       }
-      tmem_st32(tb + kColS, pk[0]);
-      tmem_st32(tb + kColS + 32, pk[1]);
+      tmem_st32(tb + kColS + out_off, pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::kBarP));
@@ -350,27 +388,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), i & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t dsk[2][32];
+      uint32_t dp[2][32];
+      tmem_ld32(tb + kColDP + 64 * g, dp[0]);
+      tmem_ld32(tb + kColDP + 64 * g + 32, dp[1]);
+      tmem_ld_wait();
+      reg_fence(dp[0]);
+      reg_fence(dp[1]);
+      uint32_t dsk[32];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t dp[32];
-        tmem_ld32(tb + kColDP + cc * 32, dp);
-        tmem_ld_wait();
-        reg_fence(dp);
-#pragma unroll
-        for (int h = 0; h < 16; ++h) {
-          const int c2 = cc * 16 + h;          // packed column
-          const int c = 2 * c2;
-          const float4 dl = *reinterpret_cast<const float4*>(st + kTileRows + (c & ~3));
-          const float d0 = (c & 2) ? dl.z : dl.x, d1 = (c & 2) ? dl.w : dl.y;
-          const uint32_t pp = pk[c2 >> 5][c2 & 31];
-          const float ds0 = bf16_lo(pp) * (__uint_as_float(dp[2 * h]) - d0);
-          const float ds1 = bf16_hi(pp) * (__uint_as_float(dp[2 * h + 1]) - d1);
-          dsk[c2 >> 5][c2 & 31] = pack_bf16(ds0, ds1);
-        }
+      for (int c2 = 0; c2 < 32; ++c2) {
+        const int c = 2 * c2;
+        const float2 dl = *reinterpret_cast<const float2*>(st + 128 + c);
+        const float ds0 = bf16_lo(pk[c2]) * (__uint_as_float(dp[c >> 5][c & 31]) - dl.x);
+        const float ds1 = bf16_hi(pk[c2]) * (__uint_as_float(dp[(c + 1) >> 5][(c + 1) & 31]) - dl.y);
+        dsk[c2] = pack_bf16(ds0, ds1);
       }
-      tmem_st32(tb + kColDP, dsk[0]);
-      tmem_st32(tb + kColDP + 32, dsk[1]);
+      tmem_st32(tb + kColDP + out_off, dsk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::kBarDS));
@@ -379,12 +412,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok) {
       raise_error(status, abort_flag, kStatusTimeout);
     } else {
+      // warpgroup 0 writes dV (into the V tile), warpgroup 1 writes dK (into the K tile)
       tc_fence_after();
       const int wrow = (warp & 3) * 32;
-      stage_row_bf16<D>(tb + kColDV, 1.f, smem + L::kOffV, r);
-      store_warp_rows<D>(&tmdV, sb + L::kOffV, wrow, kv0, bh, lane, N);
-      stage_row_bf16<D>(tb + kColDK, scale, smem + L::kOffK, r);
-      store_warp_rows<D>(&tmdK, sb + L::kOffK, wrow, kv0, bh, lane, N);
+      if (g == 0) {
+        stage_row_bf16<D>(tb + kColDV, 1.f, smem + L::kOffV, r);
+        store_warp_rows<D>(&tmdV, sb + L::kOffV, wrow, kv0, bh, lane, N);
+      } else {
+        stage_row_bf16<D>(tb + kColDK, scale, smem + L::kOffK, r);
+        store_warp_rows<D>(&tmdK, sb + L::kOffK, wrow, kv0, bh, lane, N);
+      }
     }
   }
 
@@ -399,21 +436,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ----------------------------------------------------------------------------- stage 3: dQ
 template <int D>
 struct DqSmem {
-  using T = Tiles<D>;
-  static constexpr int kStages = 2;
-  static constexpr int kOffQ = 0;                              // Q_i (later dQ staging)
-  static constexpr int kOffdO = kOffQ + T::kTile;
-  static constexpr int kOffK = kOffdO + T::kTile;              // [stage] K_j
-  static constexpr int kOffV = kOffK + kStages * T::kTile;     // [stage] V_j
-  static constexpr int kOffBar = kOffV + kStages * T::kTile;
+  using T = Tile<D, 128>;
+  static constexpr int kKStages = 2;
+  static constexpr int kVStages = (D == 128) ? 1 : 2;
+  static constexpr int kOffQ = 0;                                // Q_0, Q_1 (later dQ staging)
+  static constexpr int kOffdO = kOffQ + 2 * T::kBytes;           // dO_0, dO_1
+  static constexpr int kOffK = kOffdO + 2 * T::kBytes;           // [K stage]
+  static constexpr int kOffV = kOffK + kKStages * T::kBytes;     // [V stage]
+  static constexpr int kOffBar = kOffV + kVStages * T::kBytes;
   static constexpr int kBarQ = 0;
-  static constexpr int kBarKVFull = 1;
-  static constexpr int kBarKVEmpty = kBarKVFull + kStages;
-  static constexpr int kBarS = kBarKVEmpty + kStages;
-  static constexpr int kBarDP = kBarS + 1;
-  static constexpr int kBarDS = kBarDP + 1;
-  static constexpr int kBarAcc = kBarDS + 1;
-  static constexpr int kBarMmaDone = kBarAcc + 1;
+  static constexpr int kBarKFull = 1;
+  static constexpr int kBarKEmpty = kBarKFull + kKStages;
+  static constexpr int kBarVFull = kBarKEmpty + kKStages;
+  static constexpr int kBarVEmpty = kBarVFull + kVStages;
+  static constexpr int kBarS = kBarVEmpty + kVStages;   // [2]
+  static constexpr int kBarSC = kBarS + 2;              // [2] S read by the softmax
+  static constexpr int kBarDP = kBarSC + 2;             // [2]
+  static constexpr int kBarDS = kBarDP + 2;             // [2]
+  static constexpr int kBarAcc = kBarDS + 2;            // [2]
+  static constexpr int kBarMmaDone = kBarAcc + 2;
   static constexpr int kNumBars = kBarMmaDone + 1;
   static constexpr int kOffSlot = kOffBar + 8 * kNumBars;
   static constexpr int kBytes = (kOffSlot + 16 + 1024) > 122880 ? (kOffSlot + 16 + 1024) : 122880;  // 1 CTA / SM
@@ -424,10 +465,10 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                  const __grid_constant__ CUtensorMap tmdQ, const float* __restrict__ lse,
-                  const float* __restrict__ delta, int N, int BH, int nt, float scale, int* status) {
+                  const __grid_constant__ CUtensorMap tmdQ, const float* __restrict__ ws_nl,
+                  const float* __restrict__ ws_delta, int N, int Npad, int BH, int nqb, float scale, int* status) {
   using L = DqSmem<D>;
-  using T = Tiles<D>;
+  using T = Tile<D, 128>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
@@ -436,29 +477,41 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Work item: query tile qt of head bh.  Causal: it meets key tiles 0..qt, so high
-  // qt are the heaviest and go first.
-  int qt, bh;
+  // Work item: 256 queries (two 128-row tiles) of head bh.  Causal: heaviest first.
+  int qblk, bh;
   if (CAUSAL) {
-    qt = nt - 1 - static_cast<int>(blockIdx.x / BH);
+    qblk = nqb - 1 - static_cast<int>(blockIdx.x / BH);
     bh = blockIdx.x % BH;
   } else {
-    qt = blockIdx.x % nt;
-    bh = blockIdx.x / nt;
+    qblk = blockIdx.x % nqb;
+    bh = blockIdx.x / nqb;
   }
-  const int q0 = qt * kTileRows;
-  const int n = CAUSAL ? qt + 1 : nt;     // key tiles visited
+  const int nkt = (N + 127) / 128;
+  int q0[2], nk[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    q0[t] = qblk * 256 + t * 128;
+    nk[t] = (q0[t] >= N) ? 0 : (CAUSAL ? min(nkt, q0[t] / 128 + 1) : nkt);
+  }
+  const int nmax = max(nk[0], nk[1]);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(L::kBarQ), 1);
-    for (int s = 0; s < L::kStages; ++s) {
-      mbar_init(bar(L::kBarKVFull + s), 1);
-      mbar_init(bar(L::kBarKVEmpty + s), 1);
+    for (int s = 0; s < L::kKStages; ++s) {
+      mbar_init(bar(L::kBarKFull + s), 1);
+      mbar_init(bar(L::kBarKEmpty + s), 1);
     }
-    mbar_init(bar(L::kBarS), 1);
-    mbar_init(bar(L::kBarDP), 1);
-    mbar_init(bar(L::kBarDS), kTileRows);
-    mbar_init(bar(L::kBarAcc), 1);
+    for (int s = 0; s < L::kVStages; ++s) {
+      mbar_init(bar(L::kBarVFull + s), 1);
+      mbar_init(bar(L::kBarVEmpty + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::kBarS + t), 1);
+      mbar_init(bar(L::kBarSC + t), 128);
+      mbar_init(bar(L::kBarDP + t), 1);
+      mbar_init(bar(L::kBarDS + t), 128);
+      mbar_init(bar(L::kBarAcc + t), 1);
+    }
     mbar_init(bar(L::kBarMmaDone), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -471,8 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
-  // Tensor memory: S / dS [0,128), dP [128,256), dQ [256,256+D)
-  constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+  // Tensor memory: S_t, then dP_t, then dS_t (bf16, first 64 columns) at 128t; dQ_t at 256 + D t.
 
   if (warp == 0) {
     if (lane == 0) {
@@ -480,152 +532,185 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       prefetch_tmap(&tmdO);
-      mbar_arrive_expect_tx(bar(L::kBarQ), 2 * T::kTile);
-      for (int c = 0; c < T::kNBox; ++c) {
-        tma_load_3d(sb + L::kOffQ + c * T::kBox, &tmQ, bar(L::kBarQ), c * 64, q0, bh);
-        tma_load_3d(sb + L::kOffdO + c * T::kBox, &tmdO, bar(L::kBarQ), c * 64, q0, bh);
-      }
-      int issued = 0;
+      uint32_t qbytes = 0;
+      for (int t = 0; t < 2; ++t)
+        if (nk[t] > 0) qbytes += 2 * T::kBytes;
+      mbar_arrive_expect_tx(bar(L::kBarQ), qbytes);
+      for (int t = 0; t < 2; ++t)
+        if (nk[t] > 0)
+          for (int c = 0; c < T::kNBox; ++c) {
+            tma_load_3d(sb + L::kOffQ + t * T::kBytes + c * T::kBox, &tmQ, bar(L::kBarQ), c * 64, q0[t], bh);
+            tma_load_3d(sb + L::kOffdO + t * T::kBytes + c * T::kBox, &tmdO, bar(L::kBarQ), c * 64, q0[t], bh);
+          }
+      int nkl = 0, nvl = 0;
       bool ok = true;
-      for (int j = 0; j < n; ++j) {
-        const int s = j % L::kStages;
-        if (!(ok = mbar_wait(bar(L::kBarKVEmpty + s), ((j / L::kStages) & 1) ^ 1, abort_flag))) break;
-        mbar_arrive_expect_tx(bar(L::kBarKVFull + s), 2 * T::kTile);
-        for (int c = 0; c < T::kNBox; ++c) {
-          tma_load_3d(sb + L::kOffK + s * T::kTile + c * T::kBox, &tmK, bar(L::kBarKVFull + s), c * 64,
-                      j * kTileRows, bh);
-          tma_load_3d(sb + L::kOffV + s * T::kTile + c * T::kBox, &tmV, bar(L::kBarKVFull + s), c * 64,
-                      j * kTileRows, bh);
-        }
-        ++issued;
+      for (int j = 0; j < nmax; ++j) {
+        const int ks = j % L::kKStages, vs = j % L::kVStages;
+        if (!(ok = mbar_wait(bar(L::kBarKEmpty + ks), ((j / L::kKStages) & 1) ^ 1, abort_flag))) break;
+        mbar_arrive_expect_tx(bar(L::kBarKFull + ks), T::kBytes);
+        for (int c = 0; c < T::kNBox; ++c)
+          tma_load_3d(sb + L::kOffK + ks * T::kBytes + c * T::kBox, &tmK, bar(L::kBarKFull + ks), c * 64, j * 128, bh);
+        ++nkl;
+        if (!(ok = mbar_wait(bar(L::kBarVEmpty + vs), ((j / L::kVStages) & 1) ^ 1, abort_flag))) break;
+        mbar_arrive_expect_tx(bar(L::kBarVFull + vs), T::kBytes);
+        for (int c = 0; c < T::kNBox; ++c)
+          tma_load_3d(sb + L::kOffV + vs * T::kBytes + c * T::kBox, &tmV, bar(L::kBarVFull + vs), c * 64, j * 128, bh);
+        ++nvl;
       }
       if (!ok) raise_error(status, abort_flag, kStatusTimeout);
       mbar_wait_drain(bar(L::kBarQ), 0);
-      for (int j = max(0, issued - L::kStages); j < issued; ++j)
-        mbar_wait_drain(bar(L::kBarKVFull + j % L::kStages), (j / L::kStages) & 1);
+      for (int j = max(0, nkl - L::kKStages); j < nkl; ++j)
+        mbar_wait_drain(bar(L::kBarKFull + j % L::kKStages), (j / L::kKStages) & 1);
+      for (int j = max(0, nvl - L::kVStages); j < nvl; ++j)
+        mbar_wait_drain(bar(L::kBarVFull + j % L::kVStages), (j / L::kVStages) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(kTileRows, kTileRows, false, false);
-      constexpr uint32_t kIdAcc = idesc_bf16(kTileRows, D, false, true);
-      const uint32_t sQ = sb + L::kOffQ, sdO = sb + L::kOffdO;
-      auto issue_s_dp = [&](int j) {
-        const uint32_t sK = sb + L::kOffK + (j % L::kStages) * T::kTile;
-        const uint32_t sV = sb + L::kOffV + (j % L::kStages) * T::kTile;
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t kIdAcc = idesc_bf16(128, D, false, true);
+      // S_t = Q_t K_j^T into region t
+      auto issue_s = [&](int t, int j) {
+        const uint32_t sQ = sb + L::kOffQ + t * T::kBytes;
+        const uint32_t sK = sb + L::kOffK + (j % L::kKStages) * T::kBytes;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * T::kBox + (kk & 3) * 32;
-          mma_ss(tmem + kColS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(sK + off, 16, 1024), kIdS, kk > 0);
-        }
-        tc_commit(bar(L::kBarS));
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * T::kBox + (kk & 3) * 32;
-          mma_ss(tmem + kColDP, sdesc_sw128(sdO + off, 16, 1024), sdesc_sw128(sV + off, 16, 1024), kIdS, kk > 0);
-        }
-        tc_commit(bar(L::kBarDP));
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + 128 * t, kmajor_desc(sQ, kk, T::kBox), kmajor_desc(sK, kk, T::kBox), kIdS, kk > 0);
+        tc_commit(bar(L::kBarS + t));
       };
       bool ok = mbar_wait(bar(L::kBarQ), 0, abort_flag);
-      for (int j = 0; ok && j < n; ++j) {
-        const int s = j % L::kStages;
-        if (j == 0) {
-          if (!(ok = mbar_wait(bar(L::kBarKVFull), 0, abort_flag))) break;
+      if (ok && nmax > 0) {
+        ok = mbar_wait(bar(L::kBarKFull), 0, abort_flag);
+        if (ok) {
           tc_fence_after();
-          issue_s_dp(0);
-        }
-        if (!(ok = mbar_wait(bar(L::kBarDS), j & 1, abort_flag))) break;
-        tc_fence_after();
-        const uint32_t sK = sb + L::kOffK + s * T::kTile;
-#pragma unroll
-        for (int kk = 0; kk < kTileRows / 16; ++kk)                       // dQ += dS K_j
-          mma_ts(tmem + kColDQ, tmem + kColS + kk * 8, sdesc_sw128(sK + kk * 2048, T::kBox, 1024), kIdAcc,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(bar(L::kBarKVEmpty + s));
-        if (j + 1 < n) {
-          const int sn = (j + 1) % L::kStages;
-          if (!(ok = mbar_wait(bar(L::kBarKVFull + sn), ((j + 1) / L::kStages) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_s_dp(j + 1);
+          for (int t = 0; t < 2; ++t)
+            if (nk[t] > 0) issue_s(t, 0);
         }
       }
+      for (int j = 0; ok && j < nmax; ++j) {
+        const int ks = j % L::kKStages, vs = j % L::kVStages;
+        const uint32_t sV = sb + L::kOffV + vs * T::kBytes;
+        const uint32_t sK = sb + L::kOffK + ks * T::kBytes;
+        bool v_ready = false;
+        for (int t = 0; t < 2 && ok; ++t) {     // dP_t = dO_t V_j^T, over S_t once it has been read
+          if (j >= nk[t]) continue;
+          if (!(ok = mbar_wait(bar(L::kBarSC + t), j & 1, abort_flag))) break;
+          if (!v_ready) {
+            if (!(ok = mbar_wait(bar(L::kBarVFull + vs), (j / L::kVStages) & 1, abort_flag))) break;
+            v_ready = true;
+          }
+          tc_fence_after();
+          const uint32_t sdO = sb + L::kOffdO + t * T::kBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            mma_ss(tmem + 128 * t, kmajor_desc(sdO, kk, T::kBox), kmajor_desc(sV, kk, T::kBox), kIdS, kk > 0);
+          tc_commit(bar(L::kBarDP + t));
+        }
+        if (!ok) break;
+        tc_commit(bar(L::kBarVEmpty + vs));
+        bool k_next = false;
+        for (int t = 0; t < 2 && ok; ++t) {     // dQ_t += dS_t K_j, then S_t for the next key tile
+          if (j >= nk[t]) continue;
+          if (!(ok = mbar_wait(bar(L::kBarDS + t), j & 1, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 128 / 16; ++kk)
+            mma_ts(tmem + 256 + D * t, tmem + 128 * t + kk * 8, mnmajor_desc(sK, kk, T::kBox), kIdAcc,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          if (j == nk[t] - 1) tc_commit(bar(L::kBarAcc + t));
+          if (j + 1 < nk[t]) {
+            if (!k_next) {
+              const int jn = j + 1;
+              if (!(ok = mbar_wait(bar(L::kBarKFull + jn % L::kKStages), (jn / L::kKStages) & 1, abort_flag)))
+                break;
+              tc_fence_after();
+              k_next = true;
+            }
+            issue_s(t, j + 1);
+          }
+        }
+        if (!ok) break;
+        tc_commit(bar(L::kBarKEmpty + ks));
+      }
       if (!ok) raise_error(status, abort_flag, kStatusTimeout);
-      tc_commit(bar(L::kBarAcc));
       tc_commit(bar(L::kBarMmaDone));
       mbar_wait_drain(bar(L::kBarMmaDone), 0);
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int r = threadIdx.x - 128;                                    // query row = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tb = tmem + lane_off;
-    const int qrow = q0 + r;
-    const bool row_in = qrow < N;
-    const float nlse = row_in ? -lse[static_cast<size_t>(bh) * N + qrow] * kLog2e : -CUDART_INF_F;
-    const float dl = row_in ? delta[static_cast<size_t>(bh) * N + qrow] : 0.f;
-    const float scale_log2 = scale * kLog2e;
+    const int t = (warp - 4) >> 2;
+    const int r = threadIdx.x - 128 * (1 + t);                          // query row = TMEM lane
+    const uint32_t tb = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    const uint32_t tR = tb + 128 * t;
+    const int qrow = q0[t] + r;
     bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      const int kv0 = j * kTileRows;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS), j & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sr[4][32];
-      tmem_ld32(tb + kColS, sr[0]);
-      tmem_ld32(tb + kColS + 32, sr[1]);
-      tmem_ld32(tb + kColS + 64, sr[2]);
-      tmem_ld32(tb + kColS + 96, sr[3]);
-      tmem_ld_wait();
-      reg_fence(sr[0]);
-      reg_fence(sr[1]);
-      reg_fence(sr[2]);
-      reg_fence(sr[3]);
-      // keep key columns c <= lim (causal diagonal, keys past N)
-      const int lim = min(CAUSAL ? qrow - kv0 : kTileRows - 1, N - 1 - kv0);
-      const bool edge = (CAUSAL && kv0 + kTileRows - 1 > q0) || (kv0 + kTileRows > N);
-      uint32_t pk[2][32];
+    if (nk[t] > 0) {
+      const size_t prow = static_cast<size_t>(bh) * Npad + qrow;       // < B*H*Npad: q0[t] < N <= Npad
+      const float nl = ws_nl[prow];
+      const float dl = ws_delta[prow];
+      const float scale_log2 = scale * kLog2e;
+      for (int j = 0; j < nk[t]; ++j) {
+        const int kv0 = j * 128;
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + t), j & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        // keep key columns c <= lim (causal diagonal, keys past N)
+        const int lim = min(CAUSAL ? qrow - kv0 : 127, N - 1 - kv0);
+        const bool edge = (CAUSAL && kv0 + 127 > q0[t]) || (kv0 + 128 > N);
+        uint32_t pk[64];
 #pragma unroll
-      for (int c2 = 0; c2 < kTileRows / 2; ++c2) {
-        const int c = 2 * c2;
-        float p0 = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), scale_log2, nlse));
-        float p1 = ex2_approx(fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), scale_log2, nlse));
-        if (edge) {
-          if (c > lim) p0 = 0.f;
-          if (c + 1 > lim) p1 = 0.f;
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sr[2][32];
+          tmem_ld32(tR + 64 * h, sr[0]);
+          tmem_ld32(tR + 64 * h + 32, sr[1]);
+          tmem_ld_wait();
+          reg_fence(sr[0]);
+          reg_fence(sr[1]);
+#pragma unroll
+          for (int c2 = 0; c2 < 32; ++c2) {
+            const int cl = 2 * c2, c = 64 * h + cl;
+            float p0 = ex2_approx(fmaf(__uint_as_float(sr[cl >> 5][cl & 31]), scale_log2, nl));
+            float p1 = ex2_approx(fmaf(__uint_as_float(sr[(cl + 1) >> 5][(cl + 1) & 31]), scale_log2, nl));
+            if (edge) {
+              if (c > lim) p0 = 0.f;
+              if (c + 1 > lim) p1 = 0.f;
+            }
+            pk[32 * h + c2] = pack_bf16(p0, p1);
+          }
         }
-        pk[c2 >> 5][c2 & 31] = pack_bf16(p0, p1);
-      }
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), j & 1, abort_flag));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t dsk[2][32];
+        tc_fence_before();
+        mbar_arrive(bar(L::kBarSC + t));                   // S_t has been read: dP_t may overwrite it
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP + t), j & 1, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t dp[32];
-        tmem_ld32(tb + kColDP + cc * 32, dp);
-        tmem_ld_wait();
-        reg_fence(dp);
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t dp[32];
+          tmem_ld32(tR + 32 * cc, dp);
+          tmem_ld_wait();
+          reg_fence(dp);
+          uint32_t dsk[16];
 #pragma unroll
-        for (int h = 0; h < 16; ++h) {
-          const int c2 = cc * 16 + h;
-          const uint32_t pp = pk[c2 >> 5][c2 & 31];
-          const float ds0 = bf16_lo(pp) * (__uint_as_float(dp[2 * h]) - dl);
-          const float ds1 = bf16_hi(pp) * (__uint_as_float(dp[2 * h + 1]) - dl);
-          dsk[c2 >> 5][c2 & 31] = pack_bf16(ds0, ds1);
+          for (int h2 = 0; h2 < 16; ++h2) {
+            const uint32_t pp = pk[16 * cc + h2];
+            const float ds0 = bf16_lo(pp) * (__uint_as_float(dp[2 * h2]) - dl);
+            const float ds1 = bf16_hi(pp) * (__uint_as_float(dp[2 * h2 + 1]) - dl);
+            dsk[h2] = pack_bf16(ds0, ds1);
+          }
+          // packed columns [16cc, 16cc+16) lie inside the dP columns already read
+          tmem_st16(tR + 16 * cc, dsk);
         }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::kBarDS + t));
       }
-      tmem_st32(tb + kColS, dsk[0]);
-      tmem_st32(tb + kColS + 32, dsk[1]);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(L::kBarDS));
-    }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarAcc), 0, abort_flag));
-    if (!ok) {
-      raise_error(status, abort_flag, kStatusTimeout);
-    } else {
-      tc_fence_after();
-      stage_row_bf16<D>(tb + kColDQ, scale, smem + L::kOffQ, r);
-      store_warp_rows<D>(&tmdQ, sb + L::kOffQ, (warp & 3) * 32, q0, bh, lane, N);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarAcc + t), 0, abort_flag));
+      if (!ok) {
+        raise_error(status, abort_flag, kStatusTimeout);
+      } else {
+        tc_fence_after();
+        stage_row_bf16<D>(tb + 256 + D * t, scale, smem + L::kOffQ + t * T::kBytes, r);
+        store_warp_rows<D>(&tmdQ, sb + L::kOffQ + t * T::kBytes, (warp & 3) * 32, q0[t], bh, lane, N);
+      }
     }
   }
 
@@ -638,12 +723,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int D>
-cudaError_t preprocess_impl(const void* o, const void* dO, float* delta, long long rows, cudaStream_t stream) {
-  const long long threads = rows * (D / 8);
+cudaError_t preprocess_impl(const BwdLaunch& a, cudaStream_t stream) {
+  const long long padded_rows = static_cast<long long>(a.BH) * a.Npad;
+  const long long threads = padded_rows * (D / 8);
   const long long blocks = (threads + 255) / 256;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dO), delta, rows);
+      static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse, a.ws_nl, a.ws_delta,
+      a.N, a.Npad, padded_rows);
   return cudaGetLastError();
 }
 
@@ -653,9 +740,9 @@ cudaError_t dkdv_impl(const BwdLaunch& a, cudaStream_t stream) {
   auto kern = bwd_dkdv_kernel<D, CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
   if (e != cudaSuccess) return e;
-  const int nt = (a.N + kTileRows - 1) / kTileRows;
-  kern<<<static_cast<unsigned>(nt) * a.BH, kThreads, L::kBytes, stream>>>(
-      a.tmQ, a.tmK, a.tmV, a.tmdO, a.tmdK, a.tmdV, a.lse, a.delta, a.N, a.BH, nt, a.scale, a.status);
+  const int nkt = (a.N + 127) / 128;
+  kern<<<static_cast<unsigned>(nkt) * a.BH, kThreads, L::kBytes, stream>>>(
+      a.tmQ, a.tmK, a.tmV, a.tmdO, a.tmdK, a.tmdV, a.ws_nl, a.ws_delta, a.N, a.Npad, a.BH, nkt, a.scale, a.status);
   return cudaGetLastError();
 }
 
@@ -665,17 +752,16 @@ cudaError_t dq_impl(const BwdLaunch& a, cudaStream_t stream) {
   auto kern = bwd_dq_kernel<D, CAUSAL>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
   if (e != cudaSuccess) return e;
-  const int nt = (a.N + kTileRows - 1) / kTileRows;
-  kern<<<static_cast<unsigned>(nt) * a.BH, kThreads, L::kBytes, stream>>>(
-      a.tmQ, a.tmK, a.tmV, a.tmdO, a.tmdQ, a.lse, a.delta, a.N, a.BH, nt, a.scale, a.status);
+  const int nqb = (a.N + 255) / 256;
+  kern<<<static_cast<unsigned>(nqb) * a.BH, kThreads, L::kBytes, stream>>>(
+      a.tmQ, a.tmK, a.tmV, a.tmdO, a.tmdQ, a.ws_nl, a.ws_delta, a.N, a.Npad, a.BH, nqb, a.scale, a.status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_bwd_preprocess(const void* o, const void* dO, float* delta, long long rows, int D,
-                                  cudaStream_t stream) {
-  return D == 64 ? preprocess_impl<64>(o, dO, delta, rows, stream) : preprocess_impl<128>(o, dO, delta, rows, stream);
+cudaError_t launch_bwd_preprocess(const BwdLaunch& a, cudaStream_t stream) {
+  return a.D == 64 ? preprocess_impl<64>(a, stream) : preprocess_impl<128>(a, stream);
 }
 
 cudaError_t launch_bwd_dkdv(const BwdLaunch& a, cudaStream_t stream) {

@@ -25,22 +25,24 @@ cudaError_t launch_fwd_bf16(const FwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
                            int BH, int N, int D, float scale, int causal, cudaStream_t stream);
 
-// Backward stage 1 (fa_bwd_sm100.cu): delta = rowsum(dO * O).
-cudaError_t launch_bwd_preprocess(const void* o, const void* dO, float* delta, long long rows, int D,
-                                  cudaStream_t stream);
-
-// Backward stages 2 and 3 (fa_bwd_sm100.cu).
+// Backward stages (fa_bwd_sm100.cu).  The workspace holds, per (b, h) and per row of
+// N padded up to a multiple of 128 (Npad): ws_nl = -lse * log2(e) (padding: -inf)
+// and ws_delta = rowsum(dO * O) (padding: 0).
 struct BwdLaunch {
-  CUtensorMap tmQ, tmK, tmV, tmdO;   // loads
-  CUtensorMap tmdQ, tmdK, tmdV;      // stores
+  CUtensorMap tmQ, tmK, tmV, tmdO;   // loads (query box rows: 64 for dK/dV, 128 for dQ)
+  CUtensorMap tmdQ, tmdK, tmdV;      // stores (32-row boxes)
+  const void* o;
+  const void* dO;
   const float* lse;
-  const float* delta;
-  int BH, N, D;
+  float* ws_nl;
+  float* ws_delta;
+  int BH, N, Npad, D;
   float scale;
   int causal;
   int* status;
   int num_sms;
 };
+cudaError_t launch_bwd_preprocess(const BwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_bwd_dkdv(const BwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_bwd_dq(const BwdLaunch& a, cudaStream_t stream);
 

@@ -1,7 +1,7 @@
 // fa_noalloc.cu -- fa_bwd_noalloc: the backward pass for callers that cannot allocate.
 //
-// fa_bwd needs a device workspace (the per-row term delta = rowsum(dO * O)) that the
-// caller allocates.  Some callers cannot: code that is handed only its input and
+// fa_bwd needs a device workspace (per row: -lse * log2(e) and delta = rowsum(dO * O))
+// that the caller allocates.  Some callers cannot: code that is handed only its input and
 // output buffers by a host framework which plans all device memory up front and
 // gives an operator neither a workspace nor access to an allocator.  For them this
 // entry point uses a fixed scratch array that lives in the library's own device
@@ -13,7 +13,7 @@
 // address is looked up once per device (cudaGetSymbolAddress, with that device
 // current) on the first call that runs on the device, and that address is what the
 // kernels receive.  Nothing in the scratch has to start at zero: the preprocess
-// kernel writes every delta value the later kernels read, so stale contents from an
+// kernel writes every value the later kernels read, so stale contents from an
 // earlier call are never used.  All calls share the one array, so two calls whose
 // work overlaps on the GPU (different streams, no ordering between them) race on it.
 #include <cuda_runtime.h>

@@ -26,7 +26,8 @@
  *     stream).  Every call is asynchronous on that stream; the library does no
  *     host synchronisation.
  *   - Supported: B, H, N >= 1; D in {64, 128} for bf16; D in {32, 64, 128} for
- *     fp32; Nq == Nk == N; causal in {0, 1}; B*H <= 65535*... (see fa_check).
+ *     fp32; Nq == Nk == N; causal in {0, 1}; ceil(N/256)*B*H < 2^31 (and
+ *     B*H <= 65535 for fa_fwd_f32).
  *   - Return value: FA_OK (0) or an fa_status code.  Arguments are validated
  *     before anything is launched; on an error nothing is launched and no
  *     output is touched.  Errors are never thrown across the ABI.
@@ -73,8 +74,12 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
                int B, int H, int N, int D, float scale, int causal, void* stream);
 
-/* Bytes of device workspace fa_bwd needs: the per-row term
- * delta_i = sum_d dO_id * O_id as (B,H,N) float32, rounded up to 256 bytes. */
+/* Bytes of device workspace fa_bwd needs.  With Npad = N rounded up to a
+ * multiple of 128, the workspace holds two float32 arrays of B*H*Npad rows:
+ *   [0, B*H*Npad)            nl_i    = -lse_i * log2(e)   (padding rows: -inf)
+ *   [B*H*Npad, 2*B*H*Npad)   delta_i = sum_d dO_id * O_id (padding rows: 0)
+ * i.e. 8 * B * H * Npad bytes (a multiple of 1024).  Returns 0 for an
+ * unsupported shape. */
 size_t fa_bwd_workspace_size(int B, int H, int N, int D);
 
 /* Backward, bf16 (recomputes P from lse; never stores an N x N matrix).
@@ -83,7 +88,7 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int D);
  *   lse            : (B,H,N) float32 from fa_fwd.
  *   dq, dk, dv     : (B,H,N,D) bf16, overwritten (not accumulated into).
  *   workspace      : device buffer of at least fa_bwd_workspace_size() bytes,
- *                    contents on entry ignored, clobbered on exit.
+ *                    16-byte aligned; contents on entry ignored, clobbered on exit.
  * Equivalent to fa_bwd_preprocess, then fa_bwd_dkdv and fa_bwd_dq on the
  * same stream. */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
@@ -91,20 +96,23 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
            void* workspace, size_t workspace_bytes,
            int B, int H, int N, int D, float scale, int causal, void* stream);
 
-/* Backward stage 1: delta (B,H,N) float32 = rowsum(dO * O) (fp32 arithmetic). */
-int fa_bwd_preprocess(const void* o, const void* dO, float* delta,
+/* Backward stage 1: fills the workspace (layout above) from O, dO and lse. */
+int fa_bwd_preprocess(const void* o, const void* dO, const float* lse,
+                      void* workspace, size_t workspace_bytes,
                       int B, int H, int N, int D, void* stream);
 
-/* Backward stage 2: dK, dV (bf16, overwritten).  Each key tile is owned by one
- * CTA that walks the query tiles, so dK and dV need no atomics. */
+/* Backward stage 2: dK, dV (bf16, overwritten), reading the workspace that
+ * stage 1 filled.  Each 128-key tile is owned by one CTA that walks the query
+ * rows, so dK and dV need no atomics. */
 int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
-                const float* lse, const float* delta, void* dk, void* dv,
+                const void* workspace, size_t workspace_bytes, void* dk, void* dv,
                 int B, int H, int N, int D, float scale, int causal, void* stream);
 
-/* Backward stage 3: dQ (bf16, overwritten).  Each query tile is owned by one
- * CTA that walks the key tiles, so dQ needs no atomics. */
+/* Backward stage 3: dQ (bf16, overwritten), reading the workspace that stage 1
+ * filled.  Each 256-query block is owned by one CTA that walks the key tiles,
+ * so dQ needs no atomics. */
 int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
-              const float* lse, const float* delta, void* dq,
+              const void* workspace, size_t workspace_bytes, void* dq,
               int B, int H, int N, int D, float scale, int causal, void* stream);
 
 /* Size of the fixed device scratch array that fa_bwd_noalloc uses (8 MiB). */
@@ -119,7 +127,7 @@ int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
  *   Scratch: a fixed FA_NOALLOC_SCRATCH_BYTES array in the library's own device
  *     memory (held by every GPU that loads the library until the process exits).
  *     Limit: fa_bwd_workspace_size(B, H, N, D) <= FA_NOALLOC_SCRATCH_BYTES,
- *     i.e. B*H*N <= 2,097,152 rows; larger problems return
+ *     i.e. B*H*ceil(N/128)*128 <= 1,048,576 rows; larger problems return
  *     FA_ERR_NOALLOC_CAPACITY before anything is launched.
  *   Set-up: the first call on a device looks up the array's device address
  *     (with that device current); make that first call before any stream capture.

@@ -36,9 +36,18 @@ def test_status_strings():
 
 
 def test_workspace_size():
-    assert fa.fa_bwd_workspace_size(1, 8, 65536, 128) == 8 * 65536 * 4
-    assert fa.fa_bwd_workspace_size(1, 1, 3, 64) == 256          # rounded up to 256 bytes
+    # two float32 arrays (-lse*log2 e and delta) of B*H*ceil(N/128)*128 rows
+    assert fa.fa_bwd_workspace_size(1, 8, 65536, 128) == 2 * 8 * 65536 * 4
+    assert fa.fa_bwd_workspace_size(1, 1, 3, 64) == 2 * 128 * 4
+    assert fa.fa_bwd_workspace_size(2, 3, 129, 64) == 2 * 6 * 256 * 4
     assert fa.fa_bwd_workspace_size(1, 1, 128, 96) == 0          # unsupported D
+
+
+def test_noalloc_capacity_check_needs_no_gpu():
+    lib = fa.load_library()
+    # 8 MiB scratch = 1,048,576 padded rows; one more 128-row block is rejected
+    assert lib.fa_bwd_noalloc(*([P] * 9), 1, 1, 1048576 + 1, 64, 0.1, 0, None) == 11
+    assert lib.fa_bwd_noalloc(*([P] * 9), 1, 1, 128, 80, 0.1, 0, None) == 3
 
 
 # Validation happens before any device call, so these run without a GPU.
@@ -79,9 +88,14 @@ def test_bwd_rejects_bad_arguments():
     assert lib.fa_bwd(*args[:8], U, P, ws, 1, 2, 256, 64, 0.125, 0, None) == 4
     assert lib.fa_bwd(*args[:3], Z, *args[4:], P, ws, 1, 2, 256, 64, 0.125, 0, None) == 1
     assert lib.fa_bwd(*args, P, ws, 1, 2, 256, 80, 0.125, 0, None) == 3
-    assert lib.fa_bwd_dq(P, P, P, P, P, P, Z, 1, 1, 128, 64, 0.1, 0, None) == 1
-    assert lib.fa_bwd_dkdv(P, P, P, P, P, P, P, U, 1, 1, 128, 64, 0.1, 0, None) == 4
-    assert lib.fa_bwd_preprocess(P, P, Z, 1, 1, 128, 64, None) == 1
+    ws1 = lib.fa_bwd_workspace_size(1, 1, 128, 64)
+    assert ws1 == 2 * 128 * 4
+    assert lib.fa_bwd_dq(P, P, P, P, P, ws1, Z, 1, 1, 128, 64, 0.1, 0, None) == 1
+    assert lib.fa_bwd_dkdv(P, P, P, P, P, ws1, P, U, 1, 1, 128, 64, 0.1, 0, None) == 4
+    assert lib.fa_bwd_dkdv(P, P, P, P, P, ws1 - 16, P, P, 1, 1, 128, 64, 0.1, 0, None) == 8
+    assert lib.fa_bwd_dq(P, P, P, P, U, ws1, P, 1, 1, 128, 64, 0.1, 0, None) == 4
+    assert lib.fa_bwd_preprocess(P, P, Z, P, ws1, 1, 1, 128, 64, None) == 1
+    assert lib.fa_bwd_preprocess(P, P, P, Z, ws1, 1, 1, 128, 64, None) == 8
 
 
 def test_binding_requires_cuda_tensors():

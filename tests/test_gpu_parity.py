@@ -2,6 +2,8 @@
 same seeded inputs.  Small cases that span several tiles and ragged tails come
 first; then the five workloads at full size (the long-context one on a seeded
 sample of 64 query rows and 64 key rows per head)."""
+import math
+
 import pytest
 import torch
 
@@ -91,20 +93,25 @@ def test_autograd_wrapper():
 
 def test_stage_entry_points_match_fa_bwd():
     """fa_bwd == fa_bwd_preprocess + fa_bwd_dkdv + fa_bwd_dq, bit for bit."""
-    w, (q, k, v, do) = _small(2, 2, 384, 128, True)
+    w, (q, k, v, do) = _small(2, 2, 300, 128, True)
     dev = torch.device("cuda")
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
     O, lse = fa.attention_forward(qd, kd, vd, w.softmax_scale, True)
     dq, dk, dv = fa.attention_backward(qd, kd, vd, O, lse, dod, w.softmax_scale, True)
-    delta = torch.empty_like(lse)
-    fa.fa_bwd_preprocess(O, dod, delta)
+    B, H, N, D = q.shape
+    ws = torch.full((fa.fa_bwd_workspace_size(B, H, N, D),), 0x5A, device=dev, dtype=torch.uint8)  # stale bytes
+    fa.fa_bwd_preprocess(O, dod, lse, ws)
     dq2, dk2, dv2 = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
-    fa.fa_bwd_dkdv(qd, kd, vd, dod, lse, delta, dk2, dv2, w.softmax_scale, True)
-    fa.fa_bwd_dq(qd, kd, vd, dod, lse, delta, dq2, w.softmax_scale, True)
+    fa.fa_bwd_dkdv(qd, kd, vd, dod, ws, dk2, dv2, w.softmax_scale, True)
+    fa.fa_bwd_dq(qd, kd, vd, dod, ws, dq2, w.softmax_scale, True)
     torch.cuda.synchronize()
     assert torch.equal(dq, dq2) and torch.equal(dk, dk2) and torch.equal(dv, dv2)
+    nl, delta = (x.cpu() for x in fa.workspace_views(ws, B, H, N))
     ref_delta = oracle.attention_delta(O.cpu(), do)
-    assert max_abs(delta.cpu(), ref_delta) < 1e-4
+    assert max_abs(delta[..., :N], ref_delta) < 1e-4
+    assert torch.equal(delta[..., N:], torch.zeros_like(delta[..., N:]))
+    assert max_abs(nl[..., :N], -lse.cpu().double() / math.log(2.0)) < 1e-5
+    assert torch.isinf(nl[..., N:]).all() and (nl[..., N:] < 0).all()
 
 
 def test_deterministic():
