@@ -34,6 +34,10 @@ namespace {
 
 constexpr int kThreads = 384;   // warp 0 loads, warp 1 issues MMAs, warps 4-11 compute
 constexpr float kLog2e = 1.44269504088896340736f;
+// Of every 8 pairs of exponentials, this many go to the FMA-pipe polynomial
+// (exp2_poly2) and the rest to the MUFU unit, which alone would bound the softmax.
+constexpr int kPolyPer8 = 3;
+__device__ __forceinline__ bool poly_pair(int c2) { return (c2 & 7) >= 8 - kPolyPer8; }
 
 // ----------------------------------------------------------------------------- stage 1
 template <int D>
@@ -367,18 +371,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // P^T[r][c] = exp2(s * scale * log2e + nl_c); causal: zero where key > query
       const int qc0 = q0 + 64 * g;                                       // query of this thread's column 0
       const bool diag = CAUSAL && (qc0 < key + 64);                      // some column may be masked
+      const float2 sl2 = make_float2(scale_log2, scale_log2);
       uint32_t pk[32];
 #pragma unroll
       for (int c2 = 0; c2 < 32; ++c2) {
         const int c = 2 * c2;
         const float2 nl = *reinterpret_cast<const float2*>(st + c);
-        float p0 = ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), scale_log2, nl.x));
-        float p1 = ex2_approx(fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), scale_log2, nl.y));
+        const float2 sv = make_float2(__uint_as_float(sr[c >> 5][c & 31]), __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]));
+        float2 p = exp2_pair(__ffma2_rn(sv, sl2, nl), poly_pair(c2));
         if (diag) {
-          if (key > qc0 + c) p0 = 0.f;
-          if (key > qc0 + c + 1) p1 = 0.f;
+          if (key > qc0 + c) p.x = 0.f;
+          if (key > qc0 + c + 1) p.y = 0.f;
         }
-        pk[c2] = pack_bf16(p0, p1);
+        pk[c2] = pack_bf16(p.x, p.y);
       }
       tmem_st32(tb + kColS + out_off, pk);
       tmem_st_wait();
@@ -399,9 +404,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c2 = 0; c2 < 32; ++c2) {
         const int c = 2 * c2;
         const float2 dl = *reinterpret_cast<const float2*>(st + 128 + c);
-        const float ds0 = bf16_lo(pk[c2]) * (__uint_as_float(dp[c >> 5][c & 31]) - dl.x);
-        const float ds1 = bf16_hi(pk[c2]) * (__uint_as_float(dp[(c + 1) >> 5][(c + 1) & 31]) - dl.y);
-        dsk[c2] = pack_bf16(ds0, ds1);
+        const float2 dpv = make_float2(__uint_as_float(dp[c >> 5][c & 31]), __uint_as_float(dp[(c + 1) >> 5][(c + 1) & 31]));
+        const float2 ds = __fmul2_rn(make_float2(bf16_lo(pk[c2]), bf16_hi(pk[c2])),
+                                     __ffma2_rn(dl, make_float2(-1.f, -1.f), dpv));
+        dsk[c2] = pack_bf16(ds.x, ds.y);
       }
       tmem_st32(tb + kColDP + out_off, dsk);
       tmem_st_wait();
@@ -668,13 +674,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c2 = 0; c2 < 32; ++c2) {
             const int cl = 2 * c2, c = 64 * h + cl;
-            float p0 = ex2_approx(fmaf(__uint_as_float(sr[cl >> 5][cl & 31]), scale_log2, nl));
-            float p1 = ex2_approx(fmaf(__uint_as_float(sr[(cl + 1) >> 5][(cl + 1) & 31]), scale_log2, nl));
+            const float2 sv = make_float2(__uint_as_float(sr[cl >> 5][cl & 31]), __uint_as_float(sr[(cl + 1) >> 5][(cl + 1) & 31]));
+            float2 p = exp2_pair(__ffma2_rn(sv, make_float2(scale_log2, scale_log2), make_float2(nl, nl)), poly_pair(c2));
             if (edge) {
-              if (c > lim) p0 = 0.f;
-              if (c + 1 > lim) p1 = 0.f;
+              if (c > lim) p.x = 0.f;
+              if (c + 1 > lim) p.y = 0.f;
             }
-            pk[32 * h + c2] = pack_bf16(p0, p1);
+            pk[32 * h + c2] = pack_bf16(p.x, p.y);
           }
         }
         tc_fence_before();
@@ -692,9 +698,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h2 = 0; h2 < 16; ++h2) {
             const uint32_t pp = pk[16 * cc + h2];
-            const float ds0 = bf16_lo(pp) * (__uint_as_float(dp[2 * h2]) - dl);
-            const float ds1 = bf16_hi(pp) * (__uint_as_float(dp[2 * h2 + 1]) - dl);
-            dsk[h2] = pack_bf16(ds0, ds1);
+            const float2 ds = __fmul2_rn(make_float2(bf16_lo(pp), bf16_hi(pp)),
+                                         __ffma2_rn(make_float2(dl, dl), make_float2(-1.f, -1.f),
+                                                    make_float2(__uint_as_float(dp[2 * h2]), __uint_as_float(dp[2 * h2 + 1]))));
+            dsk[h2] = pack_bf16(ds.x, ds.y);
           }
           // packed columns [16cc, 16cc+16) lie inside the dP columns already read
           tmem_st16(tR + 16 * cc, dsk);

@@ -22,6 +22,9 @@
 // O_1 [256+D, 256+2D).  P_t (bf16, two per 32-bit column) overwrites the first 64
 // columns of S_t once the scores have been read into registers.
 //
+// A fraction of the exponentials runs as a polynomial on the FMA pipe (exp2_poly2)
+// instead of the MUFU unit.
+//
 // Online-softmax detail: the running max used for the exponentials is only raised
 // when a new row max exceeds it by more than 2^8 (in exp2 units).  Numerator and
 // denominator then share the same, possibly stale, reference, so the normalised
@@ -40,6 +43,11 @@ constexpr int kBM = 128;            // query rows per tile (= TMEM lanes)
 constexpr int kBN = 128;            // keys per tile
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;
+// Of every 8 pairs of exponentials, this many go to the FMA-pipe polynomial
+// (exp2_poly2) and the rest to the MUFU unit.  At D = 64 the matrix products are
+// half as long, so more of the exponentials move off the MUFU.
+template <int D>
+__device__ __forceinline__ bool poly_pair(int c2) { return (c2 & 7) >= (D == 64 ? 4 : 5); }
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D>
@@ -267,7 +275,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float mx[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-      for (int c = 0; c < kBN; ++c) mx[c & 3] = fmaxf(mx[c & 3], __uint_as_float(sr[c >> 5][c & 31]));
+      for (int c = 0; c < kBN; c += 2)
+        mx[(c >> 1) & 3] = fmax3(mx[(c >> 1) & 3], __uint_as_float(sr[c >> 5][c & 31]),
+                                 __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]));
       const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * scale_log2;
       const float m_new = fmaxf(m, m_tile);
       const bool need = m_new > m + kRescaleThreshold;                     // always true at j == 0
@@ -275,16 +285,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float alpha = need ? ex2_approx(m - m_new) : 1.f;
       const float neg = (m_use == -CUDART_INF_F) ? 0.f : -m_use;
       uint32_t pk[2][32];
-      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 sum[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      const float2 sl2 = make_float2(scale_log2, scale_log2), neg2 = make_float2(neg, neg);
 #pragma unroll
       for (int c = 0; c < kBN / 2; ++c) {
-        const float p0 = ex2_approx(fmaf(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]), scale_log2, neg));
-        const float p1 = ex2_approx(fmaf(__uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]), scale_log2, neg));
-        sum[(2 * c) & 3] += p0;
-        sum[(2 * c + 1) & 3] += p1;
-        pk[c >> 5][c & 31] = pack_bf16(p0, p1);
+        const float2 sv = make_float2(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]),
+                                      __uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]));
+        const float2 p = exp2_pair(__ffma2_rn(sv, sl2, neg2), poly_pair<D>(c));
+        sum[c & 1] = __fadd2_rn(sum[c & 1], p);
+        pk[c >> 5][c & 31] = pack_bf16(p.x, p.y);
       }
-      l = l * alpha + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+      l = l * alpha + ((sum[0].x + sum[0].y) + (sum[1].x + sum[1].y));
       m = m_use;
       tmem_st32(tS, pk[0]);
       tmem_st32(tS + 32, pk[1]);
@@ -298,7 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld_wait();
           reg_fence(o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int i = 0; i < 32; i += 2) {
+            const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
+                                        make_float2(alpha, alpha));
+            o[i] = __float_as_uint(v.x);
+            o[i + 1] = __float_as_uint(v.y);
+          }
           tmem_st32(tO + cc * 32, o);
         }
       }

@@ -221,10 +221,45 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x for two values at once on the FMA pipe (packed fp32x2 arithmetic), so that part
+// of the exponentials can bypass the MUFU unit.  Cody-Waite range reduction
+// (x = n + f, n = round(x) via the 1.5*2^23 rounding trick, f in [-1/2, 1/2]), a cubic
+// for 2^f whose coefficients minimise the maximum relative error on [-1/2, 1/2]
+// (Remez exchange; derived by gen_exp2_poly.py in this directory), and 2^n applied
+// by adding n to the exponent field.  Max relative error 7.8e-5 for x in [-125, 10];
+// x below -125 (including -inf) is clamped to -125, i.e. a result of ~2.4e-38.
+constexpr float kExp2C0 = 0.99992805719375610f;   // 0x3f7ffb49
+constexpr float kExp2C1 = 0.69326096773147583f;   // 0x3f31798d
+constexpr float kExp2C2 = 0.24261112511157990f;   // 0x3e786f0d
+constexpr float kExp2C3 = 0.05517166852951050f;   // 0x3d61fbb0
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
+  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(f, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
+  p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
+  p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+// 2^x for a pair: on the FMA pipe when `poly`, else two MUFU ex2.approx.
+__device__ __forceinline__ float2 exp2_pair(float2 x, bool poly) {
+  return poly ? exp2_poly2(x) : make_float2(ex2_approx(x.x), ex2_approx(x.y));
+}
+
 // Packs two floats to bf16x2 (round to nearest even); `lo` lands in the low half.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
 
