@@ -14,7 +14,7 @@
 //                   (padding rows: nl = -inf so their P is 0, delta = 0)
 //   2. dkdv kernel  one CTA per 128-key tile walks the query tiles (128 rows):
 //                     S^T = K_j Q_i^T, dP^T = V_j dO_i^T      (M=128 keys, N=128 queries)
-//                     P^T, dS^T computed by 256 threads (a key row, half the queries each)
+//                     P^T, dS^T computed by 512 threads (a key row, a quarter of the queries each)
 //                     dV_j += P^T dO_i, dK_j += dS^T Q_i        (A operand read from TMEM)
 //                   S^T of the next query tile is computed while dS^T of this one is.
 //   3. dq kernel    one CTA per 256 queries (two 128-row tiles) walks the key tiles:
@@ -32,7 +32,10 @@
 namespace fa {
 namespace {
 
-constexpr int kThreads = 384;   // warp 0 loads, warp 1 issues MMAs, warps 4-11 compute
+// 640 threads: warp 0 loads, warp 1 issues MMAs, warps 4-19 are four warpgroups that
+// share the element-wise work (no row reduction is needed in the backward, so the
+// columns of a tile can be split across warpgroups to hide more latency).
+constexpr int kThreads = 640;
 constexpr float kLog2e = 1.44269504088896340736f;
 // Of every 8 pairs of exponentials, this many go to the FMA-pipe polynomial
 // (exp2_poly2) and the rest to the MUFU unit, which alone would bound the softmax.
@@ -83,17 +86,17 @@ struct Tile {
   static constexpr int kBytes = kBox * kNBox;
 };
 
-// Copies this thread's accumulator row (D fp32 columns of tensor memory, times `mul`)
-// as bf16 into row r of a 128-row staging tile in the TMA 128-byte-swizzled layout.
+// Copies 64 columns (box `box`) of this thread's fp32 accumulator row in tensor memory,
+// times `mul`, as bf16 into row r of that box of a 128-row staging tile in the TMA
+// 128-byte-swizzled layout.
 template <int D>
-__device__ __forceinline__ void stage_row_bf16(uint32_t tacc, float mul, uint8_t* stage, int r) {
+__device__ __forceinline__ void stage_box_bf16(uint32_t tacc, int box, float mul, uint8_t* stage, int r) {
 #pragma unroll
-  for (int cc = 0; cc < D / 32; ++cc) {
+  for (int cc = 2 * box; cc < 2 * box + 2; ++cc) {
     uint32_t o[32];
     tmem_ld32(tacc + cc * 32, o);
     tmem_ld_wait();
     reg_fence(o);
-    const int box = cc >> 1;
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
       const int chunk = (cc & 1) * 4 + q4;
@@ -107,16 +110,15 @@ __device__ __forceinline__ void stage_row_bf16(uint32_t tacc, float mul, uint8_t
   }
 }
 
-// One warp stores its 32 staged rows with the TMA (tensor map box: 64 x 32 x 1);
-// rows at or past n_rows are skipped (or clipped by the hardware).
+// One warp stores its 32 staged rows of box `box` with the TMA (tensor map box:
+// 64 x 32 x 1); rows at or past n_rows are skipped (or clipped by the hardware).
 template <int D>
-__device__ __forceinline__ void store_warp_rows(const CUtensorMap* tm, uint32_t stage_s, int wrow, int row0, int bh,
-                                                int lane, int n_rows) {
+__device__ __forceinline__ void store_warp_box(const CUtensorMap* tm, uint32_t stage_s, int box, int wrow, int row0,
+                                               int bh, int lane, int n_rows) {
   fence_async_smem();
   __syncwarp();
   if (lane == 0 && row0 + wrow < n_rows) {
-    for (int c = 0; c < Tile<D, 128>::kNBox; ++c)
-      tma_store_3d(tm, stage_s + c * Tile<D, 128>::kBox + wrow * 128, c * 64, row0 + wrow, bh);
+    tma_store_3d(tm, stage_s + box * Tile<D, 128>::kBox + wrow * 128, box * 64, row0 + wrow, bh);
     bulk_commit();
     bulk_wait_read0();
   }
@@ -139,10 +141,10 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk, int box)
 // ----------------------------------------------------------------------------- stage 2: dK, dV
 // One CTA per 128-key tile walks the query tiles (128 rows each).  Every MMA is
 // M=128 x N=128 (or N=D): S^T and dP^T (shared-memory operands), dV and dK (A from
-// tensor memory).  Two warpgroups split the 128 query columns of S^T / dP^T (64
-// each); each writes its bf16 P^T / dS^T only into columns it has already read
-// (warpgroup 0: the first 32 of its range, warpgroup 1: the last 32), and the
-// K-step addresses of the dV / dK MMAs stitch the two halves back together.
+// tensor memory).  Four warpgroups split the 128 query columns of S^T / dP^T (32
+// each); each writes its 16 columns of packed bf16 P^T / dS^T into the first half of
+// its own (already read) column range, and the K-step addresses of the dV / dK MMAs
+// stitch the four quarters back together.
 // Q and dO have separate 2-stage rings, each released right after its last use.
 template <int D>
 struct DkdvSmem {
@@ -172,11 +174,11 @@ struct DkdvSmem {
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
-// Tensor-memory column of the packed bf16 pair for K-step kk (16 queries) of the
-// P^T (base 0) or dS^T (base 128) operand: queries 0-63 at base + [0, 32),
-// queries 64-127 at base + [96, 128).
+// Tensor-memory column of the packed bf16 pairs for K-step kk (16 queries) of the
+// P^T (base 0) or dS^T (base 128) operand: queries [32g, 32g+32) are packed into
+// columns base + [32g, 32g+16).
 __device__ __forceinline__ uint32_t packed_col(uint32_t base, int kk) {
-  return base + (kk < 4 ? kk * 8 : 96 + (kk - 4) * 8);
+  return base + 32 * (kk >> 1) + 8 * (kk & 1);
 }
 
 template <int D, bool CAUSAL>
@@ -220,8 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(L::kBarS), 1);
     mbar_init(bar(L::kBarDP), 1);
-    mbar_init(bar(L::kBarP), 256);
-    mbar_init(bar(L::kBarDS), 256);
+    mbar_init(bar(L::kBarP), 512);
+    mbar_init(bar(L::kBarDS), 512);
     mbar_init(bar(L::kBarAcc), 1);
     mbar_init(bar(L::kBarMmaDone), 1);
     *abort_flag = 0;
@@ -346,38 +348,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ------------------------------------------------------------------ P^T, dS^T (64 query columns), epilogue
-    const int g = (warp - 4) >> 2;                                      // query columns [64g, 64g+64)
+    // ------------------------------------------------------------------ P^T, dS^T (32 query columns), epilogue
+    const int g = (warp - 4) >> 2;                                      // query columns [32g, 32g+32)
     const int r = threadIdx.x - 128 * (1 + g);                           // key row = TMEM lane
     const uint32_t tb = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t out_off = g == 0 ? 0 : 96;                            // where the packed half goes
     const int key = kv0 + r;
     const float scale_log2 = scale * kLog2e;
+    const float2 sl2 = make_float2(scale_log2, scale_log2);
     bool ok = true;
     for (int i = 0; i < n; ++i) {
       const int s = i % L::kStages;
       const int q0 = (it0 + i) * 128;
-      const float* st = reinterpret_cast<const float*>(smem + L::kOffStat + s * L::kStatBytes) + 64 * g;
+      const float* st = reinterpret_cast<const float*>(smem + L::kOffStat + s * L::kStatBytes) + 32 * g;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarQFull + s), (i / L::kStages) & 1, abort_flag));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS), i & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(tb + kColS + 64 * g, sr[0]);
-      tmem_ld32(tb + kColS + 64 * g + 32, sr[1]);
+      uint32_t sr[32];
+      tmem_ld32(tb + kColS + 32 * g, sr);
       tmem_ld_wait();
-      reg_fence(sr[0]);
-      reg_fence(sr[1]);
+      reg_fence(sr);
       // P^T[r][c] = exp2(s * scale * log2e + nl_c); causal: zero where key > query
-      const int qc0 = q0 + 64 * g;                                       // query of this thread's column 0
-      const bool diag = CAUSAL && (qc0 < key + 64);                      // some column may be masked
-      const float2 sl2 = make_float2(scale_log2, scale_log2);
-      uint32_t pk[32];
+      const int qc0 = q0 + 32 * g;                                       // query of this thread's column 0
+      const bool diag = CAUSAL && (qc0 < key + 32);                      // some column may be masked
+      // this warpgroup's 32 column statistics, read once (eight 16-byte loads)
+      float4 nl4[8];
 #pragma unroll
-      for (int c2 = 0; c2 < 32; ++c2) {
+      for (int q = 0; q < 8; ++q) nl4[q] = reinterpret_cast<const float4*>(st)[q];
+      uint32_t pk[16];
+#pragma unroll
+      for (int c2 = 0; c2 < 16; ++c2) {
         const int c = 2 * c2;
-        const float2 nl = *reinterpret_cast<const float2*>(st + c);
-        const float2 sv = make_float2(__uint_as_float(sr[c >> 5][c & 31]), __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]));
+        const float2 nl = (c2 & 1) ? make_float2(nl4[c2 >> 1].z, nl4[c2 >> 1].w) : make_float2(nl4[c2 >> 1].x, nl4[c2 >> 1].y);
+        const float2 sv = make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
         float2 p = exp2_pair(__ffma2_rn(sv, sl2, nl), poly_pair(c2));
         if (diag) {
           if (key > qc0 + c) p.x = 0.f;
@@ -385,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         pk[c2] = pack_bf16(p.x, p.y);
       }
-      tmem_st32(tb + kColS + out_off, pk);
+      tmem_st16(tb + kColS + 32 * g, pk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::kBarP));
@@ -393,23 +396,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), i & 1, abort_flag));
       if (!ok) break;
       tc_fence_after();
-      uint32_t dp[2][32];
-      tmem_ld32(tb + kColDP + 64 * g, dp[0]);
-      tmem_ld32(tb + kColDP + 64 * g + 32, dp[1]);
+      uint32_t dp[32];
+      tmem_ld32(tb + kColDP + 32 * g, dp);
       tmem_ld_wait();
-      reg_fence(dp[0]);
-      reg_fence(dp[1]);
-      uint32_t dsk[32];
+      reg_fence(dp);
+      float4 dl4[8];
 #pragma unroll
-      for (int c2 = 0; c2 < 32; ++c2) {
+      for (int q = 0; q < 8; ++q) dl4[q] = reinterpret_cast<const float4*>(st + 128)[q];
+      uint32_t dsk[16];
+#pragma unroll
+      for (int c2 = 0; c2 < 16; ++c2) {
         const int c = 2 * c2;
-        const float2 dl = *reinterpret_cast<const float2*>(st + 128 + c);
-        const float2 dpv = make_float2(__uint_as_float(dp[c >> 5][c & 31]), __uint_as_float(dp[(c + 1) >> 5][(c + 1) & 31]));
+        const float2 dl = (c2 & 1) ? make_float2(dl4[c2 >> 1].z, dl4[c2 >> 1].w) : make_float2(dl4[c2 >> 1].x, dl4[c2 >> 1].y);
+        const float2 dpv = make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1]));
         const float2 ds = __fmul2_rn(make_float2(bf16_lo(pk[c2]), bf16_hi(pk[c2])),
                                      __ffma2_rn(dl, make_float2(-1.f, -1.f), dpv));
         dsk[c2] = pack_bf16(ds.x, ds.y);
       }
-      tmem_st32(tb + kColDP + out_off, dsk);
+      tmem_st16(tb + kColDP + 32 * g, dsk);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::kBarDS));
@@ -418,15 +422,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok) {
       raise_error(status, abort_flag, kStatusTimeout);
     } else {
-      // warpgroup 0 writes dV (into the V tile), warpgroup 1 writes dK (into the K tile)
+      // One 64-column box per warpgroup: dV boxes into the V tile, dK boxes into the K tile.
       tc_fence_after();
       const int wrow = (warp & 3) * 32;
-      if (g == 0) {
-        stage_row_bf16<D>(tb + kColDV, 1.f, smem + L::kOffV, r);
-        store_warp_rows<D>(&tmdV, sb + L::kOffV, wrow, kv0, bh, lane, N);
-      } else {
-        stage_row_bf16<D>(tb + kColDK, scale, smem + L::kOffK, r);
-        store_warp_rows<D>(&tmdK, sb + L::kOffK, wrow, kv0, bh, lane, N);
+      const int nbox = T::kNBox;                                         // 1 (D=64) or 2 (D=128)
+      if (g < 2 * nbox) {
+        const bool is_dv = g < nbox;
+        const int box = is_dv ? g : g - nbox;
+        stage_box_bf16<D>(tb + (is_dv ? kColDV : kColDK), box, is_dv ? 1.f : scale,
+                          smem + (is_dv ? L::kOffV : L::kOffK), r);
+        store_warp_box<D>(is_dv ? &tmdV : &tmdK, sb + (is_dv ? L::kOffV : L::kOffK), box, wrow, kv0, bh, lane, N);
       }
     }
   }
@@ -513,9 +518,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(L::kBarS + t), 1);
-      mbar_init(bar(L::kBarSC + t), 128);
+      mbar_init(bar(L::kBarSC + t), 256);
       mbar_init(bar(L::kBarDP + t), 1);
-      mbar_init(bar(L::kBarDS + t), 128);
+      mbar_init(bar(L::kBarDS + t), 256);
       mbar_init(bar(L::kBarAcc + t), 1);
     }
     mbar_init(bar(L::kBarMmaDone), 1);
@@ -619,9 +624,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!(ok = mbar_wait(bar(L::kBarDS + t), j & 1, abort_flag))) break;
           tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 128 / 16; ++kk)
-            mma_ts(tmem + 256 + D * t, tmem + 128 * t + kk * 8, mnmajor_desc(sK, kk, T::kBox), kIdAcc,
-                   (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 128 / 16; ++kk)    // dQ += dS K_j; dS half h packed at 64h + [0, 32)
+            mma_ts(tmem + 256 + D * t, tmem + 128 * t + 64 * (kk >> 2) + 8 * (kk & 3),
+                   mnmajor_desc(sK, kk, T::kBox), kIdAcc, (j > 0 || kk > 0) ? 1u : 0u);
           if (j == nk[t] - 1) tc_commit(bar(L::kBarAcc + t));
           if (j + 1 < nk[t]) {
             if (!k_next) {
@@ -643,10 +648,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    const int t = (warp - 4) >> 2;
-    const int r = threadIdx.x - 128 * (1 + t);                          // query row = TMEM lane
+    // Warpgroup w = 2t + h: query tile t, key columns [64h, 64h+64) of its S / dP region;
+    // its packed bf16 dS goes to columns [64h, 64h+32) of the region.
+    const int w = (warp - 4) >> 2, t = w >> 1, h = w & 1;
+    const int r = threadIdx.x - 128 * (1 + w);                          // query row = TMEM lane
     const uint32_t tb = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    const uint32_t tR = tb + 128 * t;
+    const uint32_t tR = tb + 128 * t + 64 * h;
     const int qrow = q0[t] + r;
     bool ok = true;
     if (nk[t] > 0) {
@@ -655,32 +662,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float dl = ws_delta[prow];
       const float scale_log2 = scale * kLog2e;
       for (int j = 0; j < nk[t]; ++j) {
-        const int kv0 = j * 128;
+        const int kv0 = j * 128 + 64 * h;                               // key of this thread's column 0
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + t), j & 1, abort_flag));
         if (!ok) break;
         tc_fence_after();
         // keep key columns c <= lim (causal diagonal, keys past N)
-        const int lim = min(CAUSAL ? qrow - kv0 : 127, N - 1 - kv0);
-        const bool edge = (CAUSAL && kv0 + 127 > q0[t]) || (kv0 + 128 > N);
-        uint32_t pk[64];
+        const int lim = min(CAUSAL ? qrow - kv0 : 63, N - 1 - kv0);
+        const bool edge = lim < 63;
+        uint32_t pk[32];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sr[2][32];
-          tmem_ld32(tR + 64 * h, sr[0]);
-          tmem_ld32(tR + 64 * h + 32, sr[1]);
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t sr[32];
+          tmem_ld32(tR + 32 * hh, sr);
           tmem_ld_wait();
-          reg_fence(sr[0]);
-          reg_fence(sr[1]);
+          reg_fence(sr);
 #pragma unroll
-          for (int c2 = 0; c2 < 32; ++c2) {
-            const int cl = 2 * c2, c = 64 * h + cl;
-            const float2 sv = make_float2(__uint_as_float(sr[cl >> 5][cl & 31]), __uint_as_float(sr[(cl + 1) >> 5][(cl + 1) & 31]));
-            float2 p = exp2_pair(__ffma2_rn(sv, make_float2(scale_log2, scale_log2), make_float2(nl, nl)), poly_pair(c2));
+          for (int c2 = 0; c2 < 16; ++c2) {
+            const int cl = 2 * c2, c = 32 * hh + cl;
+            const float2 sv = make_float2(__uint_as_float(sr[cl]), __uint_as_float(sr[cl + 1]));
+            float2 p = exp2_pair(__ffma2_rn(sv, make_float2(scale_log2, scale_log2), make_float2(nl, nl)),
+                                 poly_pair(c2));
             if (edge) {
               if (c > lim) p.x = 0.f;
               if (c + 1 > lim) p.y = 0.f;
             }
-            pk[32 * h + c2] = pack_bf16(p.x, p.y);
+            pk[16 * hh + c2] = pack_bf16(p.x, p.y);
           }
         }
         tc_fence_before();
@@ -689,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t dp[32];
           tmem_ld32(tR + 32 * cc, dp);
           tmem_ld_wait();
@@ -703,7 +709,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                     make_float2(__uint_as_float(dp[2 * h2]), __uint_as_float(dp[2 * h2 + 1]))));
             dsk[h2] = pack_bf16(ds.x, ds.y);
           }
-          // packed columns [16cc, 16cc+16) lie inside the dP columns already read
+          // packed columns [16cc, 16cc+16) of this half lie inside the dP columns already read
           tmem_st16(tR + 16 * cc, dsk);
         }
         tmem_st_wait();
@@ -713,10 +719,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarAcc + t), 0, abort_flag));
       if (!ok) {
         raise_error(status, abort_flag, kStatusTimeout);
-      } else {
+      } else if (h < T::kNBox) {
+        // dQ_t box h (64 columns) into the idle Q_t tile, then TMA
         tc_fence_after();
-        stage_row_bf16<D>(tb + 256 + D * t, scale, smem + L::kOffQ + t * T::kBytes, r);
-        store_warp_rows<D>(&tmdQ, sb + L::kOffQ + t * T::kBytes, (warp & 3) * 32, q0[t], bh, lane, N);
+        stage_box_bf16<D>(tb + 256 + D * t, h, scale, smem + L::kOffQ + t * T::kBytes, r);
+        store_warp_box<D>(&tmdQ, sb + L::kOffQ + t * T::kBytes, h, (warp & 3) * 32, q0[t], bh, lane, N);
       }
     }
   }
