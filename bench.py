@@ -94,6 +94,26 @@ def recorded_traffic(kernel: str, workload: str):
     return None
 
 
+# ----------------------------------------------------------------------------- multi-rank helpers
+def shard_seed(base_seed: int, rank: int) -> int:
+    """Each rank holds its own batch/head shard of the same shape: its own input seed."""
+    return base_seed + 1000 * rank
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """The slowest rank's value (timing is max over ranks); a no-op on one rank."""
+    if world <= 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank: float, ms: float) -> float:
+    """Aggregate throughput: the work of all ranks over the slowest rank's time."""
+    return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples (every 200 ms) of one GPU while the timed region runs."""
@@ -156,7 +176,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     # each rank holds its own shard of heads: same shapes, its own seed
-    wr = workloads.custom(w.name, w.B, w.H, w.N, w.D, w.causal, dtype=w.dtype, seed=w.seed + 1000 * rank,
+    wr = workloads.custom(w.name, w.B, w.H, w.N, w.D, w.causal, dtype=w.dtype, seed=shard_seed(w.seed, rank),
                           qkv_std=w.qkv_std, scale=w.scale, backward=True)
     q_h, k_h, v_h, do_h = workloads.make_inputs(wr, with_grad_out=True)
     B, H, N, D = q_h.shape
@@ -212,10 +232,7 @@ def run_ours(args, rank, world, local_rank):
     if status != 0:
         raise RuntimeError(f"device status {status} after timed region")
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = t.item()
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
 
     # ---------------------------------------------------------------- end-to-end from host buffers
     e2e = None
@@ -236,11 +253,7 @@ def run_ours(args, rank, world, local_rank):
             _, h2d, d2h = fa.attention_fwd_bwd_from_host(*pinned, scale, causal, dev_bufs, out, stream)
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = t.item()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         e2e = {"ms_per_step": e2e_ms / args.steps, "h2d": h2d, "d2h": d2h}
     return w, per, elapsed_ms, clk.summary(), e2e
 
@@ -310,7 +323,7 @@ def main():
 
     f_fwd = w.fwd_flops()
     ms_step = elapsed_ms / args.steps
-    value = world * 2.5 * f_fwd / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(world, 2.5 * f_fwd, ms_step)
     mean = {n: statistics.mean(v) for n, v in per.items()}
     peaks, peak_kind = load_peaks()
     peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -326,7 +339,7 @@ def main():
         "t_kernels_ms": mean,
         "fwd_tflops": f_fwd / (mean["fwd"] * 1e-3) / 1e12,
         "bwd_tflops": 2.5 * f_fwd / ((mean["bwd_pre"] + mean["bwd_dkdv"] + mean["bwd_dq"]) * 1e-3) / 1e12,
-        "fwd_bwd_tflops_3_5x": world * 3.5 * f_fwd / (ms_step * 1e-3) / 1e12,
+        "fwd_bwd_tflops_3_5x": whole_job_tflops(world, 3.5 * f_fwd, ms_step),
     }
     detail["fwd_frac_of_burst_peak"] = detail["fwd_tflops"] / peak_burst
     detail["fwd_bwd_frac_of_burst_peak"] = value / world / peak_burst
@@ -353,7 +366,7 @@ def main():
         "detail": detail,
     }
     if e2e is not None:
-        out["e2e"] = {"value": world * 2.5 * f_fwd / (e2e["ms_per_step"] * 1e-3) / 1e12, "unit": "TFLOPS",
+        out["e2e"] = {"value": whole_job_tflops(world, 2.5 * f_fwd, e2e["ms_per_step"]), "unit": "TFLOPS",
                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                       "ms_per_step": e2e["ms_per_step"]}
     print(json.dumps(out))
