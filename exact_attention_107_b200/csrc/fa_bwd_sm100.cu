@@ -25,6 +25,7 @@
 // stage 3.  The probabilities used for dS are the bf16-rounded P that also feed dV.
 #include <cstdint>
 #include <math_constants.h>
+#include <type_traits>
 
 #include "fa_internal.h"
 #include "sm100_ptx.cuh"
@@ -370,24 +371,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       reg_fence(sr);
       // P^T[r][c] = exp2(s * scale * log2e + nl_c); causal: zero where key > query
       const int qc0 = q0 + 32 * g;                                       // query of this thread's column 0
-      const bool diag = CAUSAL && (qc0 < key + 32);                      // some column may be masked
+      // Warp-uniform: whether any lane of this warp has a masked column in this tile.
+      const bool diag = CAUSAL && __any_sync(0xffffffffu, qc0 < key + 32);
       // this warpgroup's 32 column statistics, read once (eight 16-byte loads)
       float4 nl4[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) nl4[q] = reinterpret_cast<const float4*>(st)[q];
       uint32_t pk[16];
+      // Two copies of the loop so that the common, unmasked tiles carry no mask tests.
+      auto p_phase = [&](auto masked) {
 #pragma unroll
-      for (int c2 = 0; c2 < 16; ++c2) {
-        const int c = 2 * c2;
-        const float2 nl = (c2 & 1) ? make_float2(nl4[c2 >> 1].z, nl4[c2 >> 1].w) : make_float2(nl4[c2 >> 1].x, nl4[c2 >> 1].y);
-        const float2 sv = make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-        float2 p = exp2_pair(__ffma2_rn(sv, sl2, nl), poly_pair(c2));
-        if (diag) {
-          if (key > qc0 + c) p.x = 0.f;
-          if (key > qc0 + c + 1) p.y = 0.f;
+        for (int c2 = 0; c2 < 16; ++c2) {
+          const int c = 2 * c2;
+          const float2 nl = (c2 & 1) ? make_float2(nl4[c2 >> 1].z, nl4[c2 >> 1].w)
+                                     : make_float2(nl4[c2 >> 1].x, nl4[c2 >> 1].y);
+          const float2 sv = make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+          float2 p = exp2_pair(__ffma2_rn(sv, sl2, nl), poly_pair(c2));
+          if (decltype(masked)::value) {
+            if (key > qc0 + c) p.x = 0.f;
+            if (key > qc0 + c + 1) p.y = 0.f;
+          }
+          pk[c2] = pack_bf16(p.x, p.y);
         }
-        pk[c2] = pack_bf16(p.x, p.y);
-      }
+      };
+      if (diag) p_phase(std::true_type{});
+      else p_phase(std::false_type{});
       tmem_st16(tb + kColS + 32 * g, pk);
       tmem_st_wait();
       tc_fence_before();
@@ -668,27 +676,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         // keep key columns c <= lim (causal diagonal, keys past N)
         const int lim = min(CAUSAL ? qrow - kv0 : 63, N - 1 - kv0);
-        const bool edge = lim < 63;
+        // Warp-uniform (the loop below contains warp-collective TMEM loads): whether any
+        // lane of this warp has a masked column in this tile.
+        const bool edge = __any_sync(0xffffffffu, lim < 63);
         uint32_t pk[32];
+        // Two copies of the loop so that the common, unmasked tiles carry no mask tests.
+        auto p_phase = [&](auto masked) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t sr[32];
-          tmem_ld32(tR + 32 * hh, sr);
-          tmem_ld_wait();
-          reg_fence(sr);
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t sr[32];
+            tmem_ld32(tR + 32 * hh, sr);
+            tmem_ld_wait();
+            reg_fence(sr);
 #pragma unroll
-          for (int c2 = 0; c2 < 16; ++c2) {
-            const int cl = 2 * c2, c = 32 * hh + cl;
-            const float2 sv = make_float2(__uint_as_float(sr[cl]), __uint_as_float(sr[cl + 1]));
-            float2 p = exp2_pair(__ffma2_rn(sv, make_float2(scale_log2, scale_log2), make_float2(nl, nl)),
-                                 poly_pair(c2));
-            if (edge) {
-              if (c > lim) p.x = 0.f;
-              if (c + 1 > lim) p.y = 0.f;
+            for (int c2 = 0; c2 < 16; ++c2) {
+              const int cl = 2 * c2, c = 32 * hh + cl;
+              const float2 sv = make_float2(__uint_as_float(sr[cl]), __uint_as_float(sr[cl + 1]));
+              float2 p = exp2_pair(__ffma2_rn(sv, make_float2(scale_log2, scale_log2), make_float2(nl, nl)),
+                                   poly_pair(c2));
+              if (decltype(masked)::value) {
+                if (c > lim) p.x = 0.f;
+                if (c + 1 > lim) p.y = 0.f;
+              }
+              pk[16 * hh + c2] = pack_bf16(p.x, p.y);
             }
-            pk[16 * hh + c2] = pack_bf16(p.x, p.y);
           }
-        }
+        };
+        if (edge) p_phase(std::true_type{});
+        else p_phase(std::false_type{});
         tc_fence_before();
         mbar_arrive(bar(L::kBarSC + t));                   // S_t has been read: dP_t may overwrite it
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP + t), j & 1, abort_flag));
