@@ -40,7 +40,7 @@ constexpr int kThreads = 640;
 constexpr float kLog2e = 1.44269504088896340736f;
 // Of every 8 pairs of exponentials, this many go to the FMA-pipe polynomial
 // (exp2_poly2) and the rest to the MUFU unit, which alone would bound the softmax.
-constexpr int kPolyPer8 = 3;
+constexpr int kPolyPer8 = 2;
 __device__ __forceinline__ bool poly_pair(int c2) { return (c2 & 7) >= 8 - kPolyPer8; }
 
 // ----------------------------------------------------------------------------- stage 1

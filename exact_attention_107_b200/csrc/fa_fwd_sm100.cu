@@ -22,9 +22,6 @@
 // O_1 [256+D, 256+2D).  P_t (bf16, two per 32-bit column) overwrites the first 64
 // columns of S_t once the scores have been read into registers.
 //
-// A fraction of the exponentials runs as a polynomial on the FMA pipe (exp2_poly2)
-// instead of the MUFU unit.
-//
 // Online-softmax detail: the running max used for the exponentials is only raised
 // when a new row max exceeds it by more than 2^8 (in exp2 units).  Numerator and
 // denominator then share the same, possibly stale, reference, so the normalised
@@ -43,11 +40,11 @@ constexpr int kBM = 128;            // query rows per tile (= TMEM lanes)
 constexpr int kBN = 128;            // keys per tile
 constexpr int kThreads = 384;
 constexpr float kRescaleThreshold = 8.0f;
-// Of every 8 pairs of exponentials, this many go to the FMA-pipe polynomial
-// (exp2_poly2) and the rest to the MUFU unit.  At D = 64 the matrix products are
-// half as long, so more of the exponentials move off the MUFU.
+// All exponentials of the forward go to the MUFU unit: with two softmax warps per SMSP
+// the FMA-pipe polynomial (exp2_poly2) gave no measurable gain here (it does in the
+// backward, whose phases run four warps per SMSP).
 template <int D>
-__device__ __forceinline__ bool poly_pair(int c2) { return (c2 & 7) >= (D == 64 ? 4 : 5); }
+__device__ __forceinline__ bool poly_pair(int) { return false; }
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D>
