@@ -1,6 +1,6 @@
 """Sequence-length sweep and standard-attention comparison on one B200.
 
-    python bench_sweep.py nsweep   [--H 8] [--D 128] [--causal 1] [--Ns 1024,2048,...]
+    python bench_sweep.py nsweep   [--H 8] [--D 128] [--causal 1] [--Ns 1024,2048,...] [--dtype fp16]
     python bench_sweep.py standard [--workload c3_bf16_fwdbwd]
 
 nsweep: for each N, forward and backward time (CUDA events, median of 5 after 2
@@ -14,7 +14,8 @@ would need more than --std-limit-gb of device memory.  Prints a markdown table.
 
 standard: the same comparison on one named workload, printing one JSON line.
 
-Inputs are seeded N(0,1) draws rounded to bf16 (the recipe of workloads.py).
+Inputs are seeded N(0,1) draws rounded to bf16, or to fp16 with --dtype fp16 (the
+recipe of workloads.py).
 """
 from __future__ import annotations
 
@@ -51,11 +52,14 @@ def fused_step(q, k, v, do, scale, causal):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, D), device=q.device, dtype=torch.uint8)
 
+    f16 = q.dtype == torch.float16
+    fwd_call, bwd_call = (fa.fa_fwd_f16, fa.fa_bwd_f16) if f16 else (fa.fa_fwd, fa.fa_bwd)
+
     def fwd():
-        fa.fa_fwd(q, k, v, o, lse, scale, causal)
+        fwd_call(q, k, v, o, lse, scale, causal)
 
     def bwd():
-        fa.fa_bwd(q, k, v, o, do, lse, dq, dk, dv, ws, scale, causal)
+        bwd_call(q, k, v, o, do, lse, dq, dk, dv, ws, scale, causal)
 
     return fwd, bwd
 
@@ -92,8 +96,8 @@ def measure(make, q, k, v, do, scale, causal):
     return t_f, t_b, peak
 
 
-def inputs(B, H, N, D, causal, seed=77):
-    w = workloads.custom("sweep", B, H, N, D, causal, seed=seed)
+def inputs(B, H, N, D, causal, seed=77, dtype="bf16"):
+    w = workloads.custom("sweep", B, H, N, D, causal, dtype=dtype, seed=seed)
     return w, [t.cuda() for t in workloads.make_inputs(w, with_grad_out=True)]
 
 
@@ -103,7 +107,7 @@ def nsweep(args):
           f"| standard fwd (ms) | standard bwd (ms) | standard peak extra memory (GiB) | speedup fwd / bwd |")
     print("|---|---|---|---|---|---|---|---|---|")
     for N in Ns:
-        w, (q, k, v, do) = inputs(args.B, args.H, N, args.D, bool(args.causal))
+        w, (q, k, v, do) = inputs(args.B, args.H, N, args.D, bool(args.causal), dtype=args.dtype)
         scale = w.softmax_scale
         ff, fb, fm = measure(fused_step, q, k, v, do, scale, w.causal)
         tfl = 2.5 * w.fwd_flops() / ((ff + fb) * 1e-3) / 1e12
@@ -145,6 +149,7 @@ def main():
     ap.add_argument("--causal", type=int, default=1)
     ap.add_argument("--Ns", default="1024,2048,4096,8192,16384,32768,65536,131072")
     ap.add_argument("--std-limit-gb", type=float, default=80.0)
+    ap.add_argument("--dtype", choices=["bf16", "fp16"], default="bf16")
     ap.add_argument("--workload", default="c3_bf16_fwdbwd")
     args = ap.parse_args()
     torch.cuda.set_device(0)

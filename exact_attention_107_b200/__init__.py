@@ -15,6 +15,7 @@ from ._binding import (  # noqa: F401
     attention_fwd_bwd_from_host,
     default_scale,
     fa_bwd,
+    fa_bwd_f16,
     fa_bwd_dkdv,
     fa_bwd_dq,
     fa_bwd_noalloc,
@@ -22,6 +23,7 @@ from ._binding import (  # noqa: F401
     fa_bwd_workspace_size,
     fa_device_status,
     fa_fwd,
+    fa_fwd_f16,
     fa_fwd_f32,
     fa_version,
     flash_attention,

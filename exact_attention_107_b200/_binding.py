@@ -20,7 +20,7 @@ LIB_PATH = pathlib.Path(__file__).resolve().with_name("libfa.so")
 SYMBOLS = (
     "fa_fwd", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess",
     "fa_bwd_dkdv", "fa_bwd_dq", "fa_status_string", "fa_device_status", "fa_version",
-    "fa_bwd_noalloc",
+    "fa_bwd_noalloc", "fa_fwd_f16", "fa_bwd_f16",
 )
 
 _lib = None
@@ -43,9 +43,11 @@ def load_library() -> ctypes.CDLL:
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_fwd_f32.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_fwd_f16.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.fa_bwd_workspace_size.restype = sz
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
+    lib.fa_bwd_f16.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
     lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, vp, sz, i, i, i, i, vp]
     lib.fa_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, sz, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_bwd_dq.argtypes = [vp, vp, vp, vp, vp, sz, vp, i, i, i, i, f, i, vp]
@@ -55,8 +57,8 @@ def load_library() -> ctypes.CDLL:
     lib.fa_status_string.restype = ctypes.c_char_p
     lib.fa_device_status.argtypes = [i]
     lib.fa_version.argtypes = []
-    for name in ("fa_fwd", "fa_fwd_f32", "fa_bwd", "fa_bwd_preprocess", "fa_bwd_dkdv", "fa_bwd_dq",
-                 "fa_device_status", "fa_version"):
+    for name in ("fa_fwd", "fa_fwd_f32", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16", "fa_bwd_preprocess", "fa_bwd_dkdv",
+                 "fa_bwd_dq", "fa_device_status", "fa_version"):
         getattr(lib, name).restype = i
     _lib = lib
     return lib
@@ -101,12 +103,21 @@ def default_scale(D: int) -> float:
 # ----------------------------------------------------------------------------- C-ABI calls
 def fa_fwd(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> None:
     """O, lse <- attention(q, k, v); bf16 (B,H,N,D) tensors, lse (B,H,N) float32."""
+    _fwd16("fa_fwd", torch.bfloat16, q, k, v, o, lse, scale, causal, stream)
+
+
+def fa_fwd_f16(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> None:
+    """O, lse <- attention(q, k, v); fp16 (B,H,N,D) tensors, lse (B,H,N) float32."""
+    _fwd16("fa_fwd_f16", torch.float16, q, k, v, o, lse, scale, causal, stream)
+
+
+def _fwd16(name, dtype, q, k, v, o, lse, scale, causal, stream) -> None:
     B, H, N, D = q.shape
-    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
-        _check(t, name, torch.bfloat16, (B, H, N, D))
+    for tn, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _check(t, tn, dtype, (B, H, N, D))
     _check(lse, "lse", torch.float32, (B, H, N))
-    _raise(load_library().fa_fwd(_p(q), _p(k), _p(v), _p(o), _p(lse), B, H, N, D, float(scale), int(causal),
-                                 _stream(stream)), "fa_fwd")
+    _raise(getattr(load_library(), name)(_p(q), _p(k), _p(v), _p(o), _p(lse), B, H, N, D, float(scale),
+                                         int(causal), _stream(stream)), name)
 
 
 def fa_fwd_f32(q, k, v, o, lse, scale: float, causal: bool, stream=None) -> None:
@@ -124,17 +135,24 @@ def fa_bwd_workspace_size(B: int, H: int, N: int, D: int) -> int:
 
 
 def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, causal: bool, stream=None) -> None:
-    """dq, dk, dv <- gradients of attention; workspace: uint8 CUDA tensor of fa_bwd_workspace_size bytes."""
+    """dq, dk, dv <- gradients of attention (bf16); workspace: uint8 CUDA tensor of
+    fa_bwd_workspace_size bytes."""
+    _bwd16("fa_bwd", torch.bfloat16, q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal, stream)
+
+
+def fa_bwd_f16(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, causal: bool, stream=None) -> None:
+    """fa_bwd with fp16 tensors (o and lse from fa_fwd_f16)."""
+    _bwd16("fa_bwd_f16", torch.float16, q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal, stream)
+
+
+def _bwd16(name, dtype, q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal, stream) -> None:
     B, H, N, D = q.shape
-    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv)):
-        _check(t, name, torch.bfloat16, (B, H, N, D))
+    for tn, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _check(t, tn, dtype, (B, H, N, D))
     _check(lse, "lse", torch.float32, (B, H, N))
-    if not (workspace.is_cuda and workspace.is_contiguous()):
-        raise ValueError("workspace must be a contiguous CUDA tensor")
-    nbytes = workspace.numel() * workspace.element_size()
-    _raise(load_library().fa_bwd(_p(q), _p(k), _p(v), _p(o), _p(do), _p(lse), _p(dq), _p(dk), _p(dv),
-                                 _p(workspace), nbytes, B, H, N, D, float(scale), int(causal), _stream(stream)),
-           "fa_bwd")
+    wp, wn = _ws(workspace)
+    _raise(getattr(load_library(), name)(_p(q), _p(k), _p(v), _p(o), _p(do), _p(lse), _p(dq), _p(dk), _p(dv),
+                                         wp, wn, B, H, N, D, float(scale), int(causal), _stream(stream)), name)
 
 
 def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, stream=None) -> None:
@@ -205,13 +223,15 @@ def fa_version() -> int:
 
 # ----------------------------------------------------------------------------- convenience API
 def attention_forward(q, k, v, scale: float | None = None, causal: bool = False, stream=None):
-    """Returns (O, lse).  bf16 inputs use the tensor-core path, float32 inputs the fp32 path."""
+    """Returns (O, lse).  bf16 and fp16 inputs use the tensor-core path, float32 inputs the fp32 path."""
     B, H, N, D = q.shape
     scale = default_scale(D) if scale is None else scale
     o = torch.empty_like(q)
     lse = torch.empty(B, H, N, device=q.device, dtype=torch.float32)
     if q.dtype == torch.float32:
         fa_fwd_f32(q, k, v, o, lse, scale, causal, stream)
+    elif q.dtype == torch.float16:
+        fa_fwd_f16(q, k, v, o, lse, scale, causal, stream)
     else:
         fa_fwd(q, k, v, o, lse, scale, causal, stream)
     return o, lse
@@ -219,13 +239,14 @@ def attention_forward(q, k, v, scale: float | None = None, causal: bool = False,
 
 def attention_backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, stream=None,
                        workspace=None):
-    """Returns (dQ, dK, dV) for bf16 inputs."""
+    """Returns (dQ, dK, dV) for bf16 or fp16 inputs."""
     B, H, N, D = q.shape
     scale = default_scale(D) if scale is None else scale
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     if workspace is None:
         workspace = torch.empty(fa_bwd_workspace_size(B, H, N, D), device=q.device, dtype=torch.uint8)
-    fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal, stream)
+    bwd = fa_bwd_f16 if q.dtype == torch.float16 else fa_bwd
+    bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal, stream)
     return dq, dk, dv
 
 
@@ -247,7 +268,7 @@ class FlashAttention(torch.autograd.Function):
 
 
 def flash_attention(q, k, v, scale: float | None = None, causal: bool = False):
-    """Differentiable exact attention on bf16 (B,H,N,D) CUDA tensors."""
+    """Differentiable exact attention on bf16 or fp16 (B,H,N,D) CUDA tensors."""
     return FlashAttention.apply(q, k, v, default_scale(q.shape[-1]) if scale is None else scale, causal)
 
 

@@ -77,15 +77,15 @@ int check_shape(int B, int H, int N, int D, bool bf16) {
   return FA_OK;
 }
 
-// 3-D (D, N, B*H) bf16 tensor map, box 64 x box_rows x 1, 128-byte swizzle.
-int make_tmap(CUtensorMap* map, const void* ptr, int BH, int N, int D, int box_rows) {
+// 3-D (D, N, B*H) bf16 (fp16 when f16) tensor map, box 64 x box_rows x 1, 128-byte swizzle.
+int make_tmap(CUtensorMap* map, const void* ptr, int BH, int N, int D, int box_rows, bool f16) {
   auto enc = encode_fn();
   if (!enc) return FA_ERR_LAUNCH;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+  const CUresult r = enc(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_LAUNCH;
@@ -133,8 +133,11 @@ int fa_device_status(int reset) {
   return v;
 }
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int D,
-           float scale, int causal, void* stream) {
+}  // extern "C"
+
+// The 16-bit paths, bf16 or (f16) fp16 operands.
+static int fwd16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int D,
+                 float scale, int causal, void* stream, bool f16) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
   int st = check_shape(B, H, N, D, true);
   if (st != FA_OK) return st;
@@ -144,10 +147,11 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   if ((st = device_state(&ds)) != FA_OK) return st;
   fa::FwdLaunch a{};
   const int BH = B * H;
-  if ((st = make_tmap(&a.tmQ, q, BH, N, D, 128)) != FA_OK) return st;
-  if ((st = make_tmap(&a.tmK, k, BH, N, D, 128)) != FA_OK) return st;
-  if ((st = make_tmap(&a.tmV, v, BH, N, D, 128)) != FA_OK) return st;
-  if ((st = make_tmap(&a.tmO, o, BH, N, D, 32)) != FA_OK) return st;
+  if ((st = make_tmap(&a.tmQ, q, BH, N, D, 128, f16)) != FA_OK) return st;
+  if ((st = make_tmap(&a.tmK, k, BH, N, D, 128, f16)) != FA_OK) return st;
+  if ((st = make_tmap(&a.tmV, v, BH, N, D, 128, f16)) != FA_OK) return st;
+  if ((st = make_tmap(&a.tmO, o, BH, N, D, 32, f16)) != FA_OK) return st;
+  a.f16 = f16 ? 1 : 0;
   a.lse = lse;
   a.BH = BH;
   a.N = N;
@@ -156,7 +160,19 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   a.causal = causal;
   a.status = ds->status;
   a.num_sms = ds->num_sms;
-  return launch_status(fa::launch_fwd_bf16(a, static_cast<cudaStream_t>(stream)));
+  return launch_status(fa::launch_fwd_16(a, static_cast<cudaStream_t>(stream)));
+}
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int D,
+           float scale, int causal, void* stream) {
+  return fwd16(q, k, v, o, lse, B, H, N, D, scale, causal, stream, false);
+}
+
+int fa_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int D,
+               float scale, int causal, void* stream) {
+  return fwd16(q, k, v, o, lse, B, H, N, D, scale, causal, stream, true);
 }
 
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B, int H, int N, int D,
@@ -189,8 +205,10 @@ static int workspace_views(void* ws, size_t ws_bytes, int B, int H, int N, int D
   return FA_OK;
 }
 
-int fa_bwd_preprocess(const void* o, const void* dO, const float* lse, void* workspace, size_t workspace_bytes,
-                      int B, int H, int N, int D, void* stream) {
+}  // extern "C"
+
+static int preprocess16(const void* o, const void* dO, const float* lse, void* workspace, size_t workspace_bytes,
+                        int B, int H, int N, int D, void* stream, bool f16) {
   if (!o || !dO || !lse) return FA_ERR_NULL;
   int st = check_shape(B, H, N, D, true);
   if (st != FA_OK) return st;
@@ -199,6 +217,7 @@ int fa_bwd_preprocess(const void* o, const void* dO, const float* lse, void* wor
   if ((st = workspace_views(workspace, workspace_bytes, B, H, N, D, &a)) != FA_OK) return st;
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
+  a.f16 = f16 ? 1 : 0;
   a.o = o;
   a.dO = dO;
   a.lse = lse;
@@ -210,7 +229,7 @@ int fa_bwd_preprocess(const void* o, const void* dO, const float* lse, void* wor
 
 static int bwd_common(const void* q, const void* k, const void* v, const void* dO, const void* workspace,
                       size_t workspace_bytes, int B, int H, int N, int D, float scale, int causal, int q_box_rows,
-                      fa::BwdLaunch* a) {
+                      bool f16, fa::BwdLaunch* a) {
   if (!q || !k || !v || !dO) return FA_ERR_NULL;
   int st = check_shape(B, H, N, D, true);
   if (st != FA_OK) return st;
@@ -220,10 +239,11 @@ static int bwd_common(const void* q, const void* k, const void* v, const void* d
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
   const int BH = B * H;
-  if ((st = make_tmap(&a->tmQ, q, BH, N, D, q_box_rows)) != FA_OK) return st;
-  if ((st = make_tmap(&a->tmK, k, BH, N, D, 128)) != FA_OK) return st;
-  if ((st = make_tmap(&a->tmV, v, BH, N, D, 128)) != FA_OK) return st;
-  if ((st = make_tmap(&a->tmdO, dO, BH, N, D, q_box_rows)) != FA_OK) return st;
+  if ((st = make_tmap(&a->tmQ, q, BH, N, D, q_box_rows, f16)) != FA_OK) return st;
+  if ((st = make_tmap(&a->tmK, k, BH, N, D, 128, f16)) != FA_OK) return st;
+  if ((st = make_tmap(&a->tmV, v, BH, N, D, 128, f16)) != FA_OK) return st;
+  if ((st = make_tmap(&a->tmdO, dO, BH, N, D, q_box_rows, f16)) != FA_OK) return st;
+  a->f16 = f16 ? 1 : 0;
   a->BH = BH;
   a->N = N;
   a->D = D;
@@ -234,33 +254,34 @@ static int bwd_common(const void* q, const void* k, const void* v, const void* d
   return FA_OK;
 }
 
-int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, const void* workspace,
-                size_t workspace_bytes, void* dk, void* dv, int B, int H, int N, int D, float scale, int causal,
-                void* stream) {
+static int dkdv16(const void* q, const void* k, const void* v, const void* dO, const void* workspace,
+                  size_t workspace_bytes, void* dk, void* dv, int B, int H, int N, int D, float scale, int causal,
+                  void* stream, bool f16) {
   if (!dk || !dv) return FA_ERR_NULL;
   if (!aligned16(dk) || !aligned16(dv)) return FA_ERR_ALIGN;
   fa::BwdLaunch a{};
-  int st = bwd_common(q, k, v, dO, workspace, workspace_bytes, B, H, N, D, scale, causal, 128, &a);
+  int st = bwd_common(q, k, v, dO, workspace, workspace_bytes, B, H, N, D, scale, causal, 128, f16, &a);
   if (st != FA_OK) return st;
-  if ((st = make_tmap(&a.tmdK, dk, a.BH, N, D, 32)) != FA_OK) return st;
-  if ((st = make_tmap(&a.tmdV, dv, a.BH, N, D, 32)) != FA_OK) return st;
+  if ((st = make_tmap(&a.tmdK, dk, a.BH, N, D, 32, f16)) != FA_OK) return st;
+  if ((st = make_tmap(&a.tmdV, dv, a.BH, N, D, 32, f16)) != FA_OK) return st;
   return launch_status(fa::launch_bwd_dkdv(a, static_cast<cudaStream_t>(stream)));
 }
 
-int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO, const void* workspace,
-              size_t workspace_bytes, void* dq, int B, int H, int N, int D, float scale, int causal, void* stream) {
+static int dq16(const void* q, const void* k, const void* v, const void* dO, const void* workspace,
+                size_t workspace_bytes, void* dq, int B, int H, int N, int D, float scale, int causal, void* stream,
+                bool f16) {
   if (!dq) return FA_ERR_NULL;
   if (!aligned16(dq)) return FA_ERR_ALIGN;
   fa::BwdLaunch a{};
-  int st = bwd_common(q, k, v, dO, workspace, workspace_bytes, B, H, N, D, scale, causal, 128, &a);
+  int st = bwd_common(q, k, v, dO, workspace, workspace_bytes, B, H, N, D, scale, causal, 128, f16, &a);
   if (st != FA_OK) return st;
-  if ((st = make_tmap(&a.tmdQ, dq, a.BH, N, D, 32)) != FA_OK) return st;
+  if ((st = make_tmap(&a.tmdQ, dq, a.BH, N, D, 32, f16)) != FA_OK) return st;
   return launch_status(fa::launch_bwd_dq(a, static_cast<cudaStream_t>(stream)));
 }
 
-int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
-           void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int D, float scale,
-           int causal, void* stream) {
+static int bwd16(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int D,
+                 float scale, int causal, void* stream, bool f16) {
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_NULL;
   int st = check_shape(B, H, N, D, true);
   if (st != FA_OK) return st;
@@ -270,11 +291,41 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
     return FA_ERR_ALIGN;
   if (!scale_ok(scale) || (causal != 0 && causal != 1)) return FA_ERR_ARG;
-  if ((st = fa_bwd_preprocess(o, dO, lse, workspace, workspace_bytes, B, H, N, D, stream)) != FA_OK) return st;
-  if ((st = fa_bwd_dkdv(q, k, v, dO, workspace, workspace_bytes, dk, dv, B, H, N, D, scale, causal, stream)) !=
+  if ((st = preprocess16(o, dO, lse, workspace, workspace_bytes, B, H, N, D, stream, f16)) != FA_OK) return st;
+  if ((st = dkdv16(q, k, v, dO, workspace, workspace_bytes, dk, dv, B, H, N, D, scale, causal, stream, f16)) !=
       FA_OK)
     return st;
-  return fa_bwd_dq(q, k, v, dO, workspace, workspace_bytes, dq, B, H, N, D, scale, causal, stream);
+  return dq16(q, k, v, dO, workspace, workspace_bytes, dq, B, H, N, D, scale, causal, stream, f16);
+}
+
+extern "C" {
+
+int fa_bwd_preprocess(const void* o, const void* dO, const float* lse, void* workspace, size_t workspace_bytes,
+                      int B, int H, int N, int D, void* stream) {
+  return preprocess16(o, dO, lse, workspace, workspace_bytes, B, H, N, D, stream, false);
+}
+
+int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, const void* workspace,
+                size_t workspace_bytes, void* dk, void* dv, int B, int H, int N, int D, float scale, int causal,
+                void* stream) {
+  return dkdv16(q, k, v, dO, workspace, workspace_bytes, dk, dv, B, H, N, D, scale, causal, stream, false);
+}
+
+int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO, const void* workspace,
+              size_t workspace_bytes, void* dq, int B, int H, int N, int D, float scale, int causal, void* stream) {
+  return dq16(q, k, v, dO, workspace, workspace_bytes, dq, B, H, N, D, scale, causal, stream, false);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
+           void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int D, float scale,
+           int causal, void* stream) {
+  return bwd16(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N, D, scale, causal, stream, false);
+}
+
+int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+               void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int D,
+               float scale, int causal, void* stream) {
+  return bwd16(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N, D, scale, causal, stream, true);
 }
 
 }  // extern "C"

@@ -1,4 +1,4 @@
-// fa_bwd_sm100.cu -- bf16 attention backward on the sm_100a tensor cores.
+// fa_bwd_sm100.cu -- bf16 / fp16 attention backward on the sm_100a tensor cores.
 //
 // The backward never stores P: it recomputes it from the saved logsumexp, as
 // "LLM paper notes #8: FlashAttention" (adg.csdn.net), section "recomputation",
@@ -22,7 +22,9 @@
 //                     read), dS, dQ_i += dS K_j
 // Every output tile is owned by exactly one CTA: no atomics, no fp32 dQ accumulator
 // in device memory, deterministic results; the price is recomputing S and dP in
-// stage 3.  The probabilities used for dS are the bf16-rounded P that also feed dV.
+// stage 3.  The probabilities used for dS are the 16-bit-rounded P that also feed dV.
+// All 16-bit operands (inputs, P, dS, outputs) take the inputs' element type: bf16,
+// or fp16 when the kernels' F16 parameter is set.
 #include <cstdint>
 #include <math_constants.h>
 #include <type_traits>
@@ -44,13 +46,13 @@ constexpr int kPolyPer8 = 2;
 __device__ __forceinline__ bool poly_pair(int c2) { return (c2 & 7) >= 8 - kPolyPer8; }
 
 // ----------------------------------------------------------------------------- stage 1
-template <int D>
-__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16* __restrict__ o,
-                                                             const __nv_bfloat16* __restrict__ dO,
+template <int D, bool F16>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint16_t* __restrict__ o,
+                                                             const uint16_t* __restrict__ dO,
                                                              const float* __restrict__ lse,
                                                              float* __restrict__ ws_nl, float* __restrict__ ws_delta,
                                                              int N, int Npad, long long padded_rows) {
-  constexpr int kLanesPerRow = D / 8;   // each lane reads 8 bf16 (16 bytes) of O and of dO
+  constexpr int kLanesPerRow = D / 8;   // each lane reads 8 values (16 bytes) of O and of dO
   const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long prow = gt / kLanesPerRow;          // row in the padded (B*H, Npad) layout
   const int part = static_cast<int>(gt % kLanesPerRow);
@@ -65,8 +67,8 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16
     const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      acc = fmaf(__uint_as_float(av[i] << 16), __uint_as_float(bv[i] << 16), acc);
-      acc = fmaf(__uint_as_float(av[i] & 0xffff0000u), __uint_as_float(bv[i] & 0xffff0000u), acc);
+      acc = fmaf(unpack16_lo<F16>(av[i]), unpack16_lo<F16>(bv[i]), acc);
+      acc = fmaf(unpack16_hi<F16>(av[i]), unpack16_hi<F16>(bv[i]), acc);
     }
   }
 #pragma unroll
@@ -78,7 +80,7 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const __nv_bfloat16
 }
 
 // ----------------------------------------------------------------------------- shared helpers
-// A tile of `rows` rows x D bf16 in shared memory, stored as D/64 boxes of rows x 128 bytes
+// A tile of `rows` rows x D 16-bit values in shared memory, stored as D/64 boxes of rows x 128 bytes
 // in the TMA 128-byte-swizzled layout.
 template <int D, int ROWS>
 struct Tile {
@@ -88,10 +90,10 @@ struct Tile {
 };
 
 // Copies 64 columns (box `box`) of this thread's fp32 accumulator row in tensor memory,
-// times `mul`, as bf16 into row r of that box of a 128-row staging tile in the TMA
+// times `mul`, as bf16 (fp16 when F16) into row r of that box of a 128-row staging tile in the TMA
 // 128-byte-swizzled layout.
-template <int D>
-__device__ __forceinline__ void stage_box_bf16(uint32_t tacc, int box, float mul, uint8_t* stage, int r) {
+template <int D, bool F16>
+__device__ __forceinline__ void stage_box_16(uint32_t tacc, int box, float mul, uint8_t* stage, int r) {
 #pragma unroll
   for (int cc = 2 * box; cc < 2 * box + 2; ++cc) {
     uint32_t o[32];
@@ -102,10 +104,10 @@ __device__ __forceinline__ void stage_box_bf16(uint32_t tacc, int box, float mul
     for (int q4 = 0; q4 < 4; ++q4) {
       const int chunk = (cc & 1) * 4 + q4;
       uint4 v;
-      v.x = pack_bf16(__uint_as_float(o[8 * q4 + 0]) * mul, __uint_as_float(o[8 * q4 + 1]) * mul);
-      v.y = pack_bf16(__uint_as_float(o[8 * q4 + 2]) * mul, __uint_as_float(o[8 * q4 + 3]) * mul);
-      v.z = pack_bf16(__uint_as_float(o[8 * q4 + 4]) * mul, __uint_as_float(o[8 * q4 + 5]) * mul);
-      v.w = pack_bf16(__uint_as_float(o[8 * q4 + 6]) * mul, __uint_as_float(o[8 * q4 + 7]) * mul);
+      v.x = pack16<F16>(__uint_as_float(o[8 * q4 + 0]) * mul, __uint_as_float(o[8 * q4 + 1]) * mul);
+      v.y = pack16<F16>(__uint_as_float(o[8 * q4 + 2]) * mul, __uint_as_float(o[8 * q4 + 3]) * mul);
+      v.z = pack16<F16>(__uint_as_float(o[8 * q4 + 4]) * mul, __uint_as_float(o[8 * q4 + 5]) * mul);
+      v.w = pack16<F16>(__uint_as_float(o[8 * q4 + 6]) * mul, __uint_as_float(o[8 * q4 + 7]) * mul);
       *reinterpret_cast<uint4*>(stage + box * Tile<D, 128>::kBox + r * 128 + ((chunk ^ (r & 7)) << 4)) = v;
     }
   }
@@ -126,10 +128,7 @@ __device__ __forceinline__ void store_warp_box(const CUtensorMap* tm, uint32_t s
   __syncwarp();
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
-
-// K-major operand slice for K-step kk (16 bf16 = 32 bytes) of a swizzled tile with box size `box`.
+// K-major operand slice for K-step kk (16 values = 32 bytes) of a swizzled tile with box size `box`.
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk, int box) {
   return sdesc_sw128(tile + (kk >> 2) * box + (kk & 3) * 32, 16, 1024);
 }
@@ -143,7 +142,7 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk, int box)
 // One CTA per 128-key tile walks the query tiles (128 rows each).  Every MMA is
 // M=128 x N=128 (or N=D): S^T and dP^T (shared-memory operands), dV and dK (A from
 // tensor memory).  Four warpgroups split the 128 query columns of S^T / dP^T (32
-// each); each writes its 16 columns of packed bf16 P^T / dS^T into the first half of
+// each); each writes its 16 columns of packed 16-bit P^T / dS^T into the first half of
 // its own (already read) column range, and the K-step addresses of the dV / dK MMAs
 // stitch the four quarters back together.
 // Q and dO have separate 2-stage rings, each released right after its last use.
@@ -175,14 +174,14 @@ struct DkdvSmem {
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
-// Tensor-memory column of the packed bf16 pairs for K-step kk (16 queries) of the
+// Tensor-memory column of the packed 16-bit pairs for K-step kk (16 queries) of the
 // P^T (base 0) or dS^T (base 128) operand: queries [32g, 32g+32) are packed into
 // columns base + [32g, 32g+16).
 __device__ __forceinline__ uint32_t packed_col(uint32_t base, int kk) {
   return base + 32 * (kk >> 1) + 8 * (kk & 1);
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -286,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);   // S^T, dP^T: K-major A and B
-      constexpr uint32_t kIdAcc = idesc_bf16(128, D, false, true);    // dV, dK: A in TMEM, B MN-major
+      constexpr uint32_t kIdS = idesc_16(128, 128, false, false, F16);  // S^T, dP^T: K-major A and B
+      constexpr uint32_t kIdAcc = idesc_16(128, D, false, true, F16);   // dV, dK: A in TMEM, B MN-major
       const uint32_t sK = sb + L::kOffK, sV = sb + L::kOffV;
       auto issue_st = [&](int i) {      // S^T = K_j Q_i^T
         const uint32_t sQ = sb + L::kOffQ + (i % L::kStages) * T::kBytes;
@@ -303,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tmem + kColDP, kmajor_desc(sV, kk, T::kBox), kmajor_desc(sdO, kk, T::kBox), kIdS, kk > 0);
         tc_commit(bar(L::kBarDP));
       };
-      // acc (+)= A_tmem (packed bf16, 128 queries) * B_smem (128 queries x D, MN-major)
+      // acc (+)= A_tmem (packed 16-bit, 128 queries) * B_smem (128 queries x D, MN-major)
       auto issue_acc = [&](uint32_t dcol, uint32_t abase, uint32_t b_tile, bool first) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -391,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (key > qc0 + c) p.x = 0.f;
             if (key > qc0 + c + 1) p.y = 0.f;
           }
-          pk[c2] = pack_bf16(p.x, p.y);
+          pk[c2] = pack16<F16>(p.x, p.y);
         }
       };
       if (diag) p_phase(std::true_type{});
@@ -417,9 +416,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c = 2 * c2;
         const float2 dl = (c2 & 1) ? make_float2(dl4[c2 >> 1].z, dl4[c2 >> 1].w) : make_float2(dl4[c2 >> 1].x, dl4[c2 >> 1].y);
         const float2 dpv = make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1]));
-        const float2 ds = __fmul2_rn(make_float2(bf16_lo(pk[c2]), bf16_hi(pk[c2])),
+        const float2 ds = __fmul2_rn(make_float2(unpack16_lo<F16>(pk[c2]), unpack16_hi<F16>(pk[c2])),
                                      __ffma2_rn(dl, make_float2(-1.f, -1.f), dpv));
-        dsk[c2] = pack_bf16(ds.x, ds.y);
+        dsk[c2] = pack16<F16>(ds.x, ds.y);
       }
       tmem_st16(tb + kColDP + 32 * g, dsk);
       tmem_st_wait();
@@ -437,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (g < 2 * nbox) {
         const bool is_dv = g < nbox;
         const int box = is_dv ? g : g - nbox;
-        stage_box_bf16<D>(tb + (is_dv ? kColDV : kColDK), box, is_dv ? 1.f : scale,
+        stage_box_16<D, F16>(tb + (is_dv ? kColDV : kColDK), box, is_dv ? 1.f : scale,
                           smem + (is_dv ? L::kOffV : L::kOffK), r);
         store_warp_box<D>(is_dv ? &tmdV : &tmdK, sb + (is_dv ? L::kOffV : L::kOffK), box, wrow, kv0, bh, lane, N);
       }
@@ -480,7 +479,7 @@ struct DqSmem {
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -543,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
-  // Tensor memory: S_t, then dP_t, then dS_t (bf16, first 64 columns) at 128t; dQ_t at 256 + D t.
+  // Tensor memory: S_t, then dP_t, then dS_t (16-bit, first 64 columns) at 128t; dQ_t at 256 + D t.
 
   if (warp == 0) {
     if (lane == 0) {
@@ -585,8 +584,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);
-      constexpr uint32_t kIdAcc = idesc_bf16(128, D, false, true);
+      constexpr uint32_t kIdS = idesc_16(128, 128, false, false, F16);
+      constexpr uint32_t kIdAcc = idesc_16(128, D, false, true, F16);
       // S_t = Q_t K_j^T into region t
       auto issue_s = [&](int t, int j) {
         const uint32_t sQ = sb + L::kOffQ + t * T::kBytes;
@@ -657,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // Warpgroup w = 2t + h: query tile t, key columns [64h, 64h+64) of its S / dP region;
-    // its packed bf16 dS goes to columns [64h, 64h+32) of the region.
+    // its packed 16-bit dS goes to columns [64h, 64h+32) of the region.
     const int w = (warp - 4) >> 2, t = w >> 1, h = w & 1;
     const int r = threadIdx.x - 128 * (1 + w);                          // query row = TMEM lane
     const uint32_t tb = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -698,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (c > lim) p.x = 0.f;
                 if (c + 1 > lim) p.y = 0.f;
               }
-              pk[16 * hh + c2] = pack_bf16(p.x, p.y);
+              pk[16 * hh + c2] = pack16<F16>(p.x, p.y);
             }
           }
         };
@@ -719,10 +718,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int h2 = 0; h2 < 16; ++h2) {
             const uint32_t pp = pk[16 * cc + h2];
-            const float2 ds = __fmul2_rn(make_float2(bf16_lo(pp), bf16_hi(pp)),
+            const float2 ds = __fmul2_rn(make_float2(unpack16_lo<F16>(pp), unpack16_hi<F16>(pp)),
                                          __ffma2_rn(make_float2(dl, dl), make_float2(-1.f, -1.f),
                                                     make_float2(__uint_as_float(dp[2 * h2]), __uint_as_float(dp[2 * h2 + 1]))));
-            dsk[h2] = pack_bf16(ds.x, ds.y);
+            dsk[h2] = pack16<F16>(ds.x, ds.y);
           }
           // packed columns [16cc, 16cc+16) of this half lie inside the dP columns already read
           tmem_st16(tR + 16 * cc, dsk);
@@ -737,7 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (h < T::kNBox) {
         // dQ_t box h (64 columns) into the idle Q_t tile, then TMA
         tc_fence_after();
-        stage_box_bf16<D>(tb + 256 + D * t, h, scale, smem + L::kOffQ + t * T::kBytes, r);
+        stage_box_16<D, F16>(tb + 256 + D * t, h, scale, smem + L::kOffQ + t * T::kBytes, r);
         store_warp_box<D>(&tmdQ, sb + L::kOffQ + t * T::kBytes, h, (warp & 3) * 32, q0[t], bh, lane, N);
       }
     }
@@ -751,22 +750,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool F16>
 cudaError_t preprocess_impl(const BwdLaunch& a, cudaStream_t stream) {
   const long long padded_rows = static_cast<long long>(a.BH) * a.Npad;
   const long long threads = padded_rows * (D / 8);
   const long long blocks = (threads + 255) / 256;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dO), a.lse, a.ws_nl, a.ws_delta,
+  bwd_preprocess_kernel<D, F16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+      static_cast<const uint16_t*>(a.o), static_cast<const uint16_t*>(a.dO), a.lse, a.ws_nl, a.ws_delta,
       a.N, a.Npad, padded_rows);
   return cudaGetLastError();
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F16>
 cudaError_t dkdv_impl(const BwdLaunch& a, cudaStream_t stream) {
   using L = DkdvSmem<D>;
-  auto kern = bwd_dkdv_kernel<D, CAUSAL>;
+  auto kern = bwd_dkdv_kernel<D, CAUSAL, F16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
   if (e != cudaSuccess) return e;
   const int nkt = (a.N + 127) / 128;
@@ -775,10 +774,10 @@ cudaError_t dkdv_impl(const BwdLaunch& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F16>
 cudaError_t dq_impl(const BwdLaunch& a, cudaStream_t stream) {
   using L = DqSmem<D>;
-  auto kern = bwd_dq_kernel<D, CAUSAL>;
+  auto kern = bwd_dq_kernel<D, CAUSAL, F16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
   if (e != cudaSuccess) return e;
   const int nqb = (a.N + 255) / 256;
@@ -787,20 +786,35 @@ cudaError_t dq_impl(const BwdLaunch& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <bool F16>
+cudaError_t preprocess_typed(const BwdLaunch& a, cudaStream_t stream) {
+  return a.D == 64 ? preprocess_impl<64, F16>(a, stream) : preprocess_impl<128, F16>(a, stream);
+}
+
+template <bool F16>
+cudaError_t dkdv_typed(const BwdLaunch& a, cudaStream_t stream) {
+  if (a.D == 64) return a.causal ? dkdv_impl<64, true, F16>(a, stream) : dkdv_impl<64, false, F16>(a, stream);
+  return a.causal ? dkdv_impl<128, true, F16>(a, stream) : dkdv_impl<128, false, F16>(a, stream);
+}
+
+template <bool F16>
+cudaError_t dq_typed(const BwdLaunch& a, cudaStream_t stream) {
+  if (a.D == 64) return a.causal ? dq_impl<64, true, F16>(a, stream) : dq_impl<64, false, F16>(a, stream);
+  return a.causal ? dq_impl<128, true, F16>(a, stream) : dq_impl<128, false, F16>(a, stream);
+}
+
 }  // namespace
 
 cudaError_t launch_bwd_preprocess(const BwdLaunch& a, cudaStream_t stream) {
-  return a.D == 64 ? preprocess_impl<64>(a, stream) : preprocess_impl<128>(a, stream);
+  return a.f16 ? preprocess_typed<true>(a, stream) : preprocess_typed<false>(a, stream);
 }
 
 cudaError_t launch_bwd_dkdv(const BwdLaunch& a, cudaStream_t stream) {
-  if (a.D == 64) return a.causal ? dkdv_impl<64, true>(a, stream) : dkdv_impl<64, false>(a, stream);
-  return a.causal ? dkdv_impl<128, true>(a, stream) : dkdv_impl<128, false>(a, stream);
+  return a.f16 ? dkdv_typed<true>(a, stream) : dkdv_typed<false>(a, stream);
 }
 
 cudaError_t launch_bwd_dq(const BwdLaunch& a, cudaStream_t stream) {
-  if (a.D == 64) return a.causal ? dq_impl<64, true>(a, stream) : dq_impl<64, false>(a, stream);
-  return a.causal ? dq_impl<128, true>(a, stream) : dq_impl<128, false>(a, stream);
+  return a.f16 ? dq_typed<true>(a, stream) : dq_typed<false>(a, stream);
 }
 
 }  // namespace fa

@@ -1,4 +1,4 @@
-// fa_fwd_sm100.cu -- bf16 attention forward on the sm_100a tensor cores.
+// fa_fwd_sm100.cu -- bf16 / fp16 attention forward on the sm_100a tensor cores.
 //
 // Computes O = softmax(scale * Q K^T [causal]) V and lse = ln(sum_j exp(scale * q.k_j))
 // with the tiled, online-softmax scheme of "LLM paper notes #8: FlashAttention"
@@ -19,8 +19,10 @@
 // so one tile's softmax overlaps the other tile's matrix products.
 //
 // Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,256+D),
-// O_1 [256+D, 256+2D).  P_t (bf16, two per 32-bit column) overwrites the first 64
-// columns of S_t once the scores have been read into registers.
+// O_1 [256+D, 256+2D).  P_t (16-bit, two per 32-bit column) overwrites the first 64
+// columns of S_t once the scores have been read into registers.  P_t takes the
+// element type of the inputs (bf16, or fp16 when F16), as the tensor-core operands
+// of one MMA share one type.
 //
 // Online-softmax detail: the running max used for the exponentials is only raised
 // when a new row max exceeds it by more than 2^8 (in exp2 units).  Numerator and
@@ -50,7 +52,7 @@ constexpr float kLn2 = 0.69314718055994530942f;
 template <int D>
 struct FwdSmem {
   static constexpr int kStages = (D == 128) ? 2 : 4;
-  static constexpr int kBox = 128 * 64 * 2;      // 128 rows x 64 bf16: one 128-byte swizzle span
+  static constexpr int kBox = 128 * 64 * 2;      // 128 rows x 64 16-bit values: one 128-byte swizzle span
   static constexpr int kNBox = D / 64;
   static constexpr int kTile = kBox * kNBox;     // one 128-row tile of Q, K, V (or O staging)
   static constexpr int kOffQ = 0;                // 2 query tiles (reused to stage O)
@@ -74,9 +76,9 @@ struct FwdSmem {
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
-    fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                     float* __restrict__ lse, int N, int BH, int nqb, float scale_log2, int* status) {
   using L = FwdSmem<D>;
@@ -176,8 +178,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(kBM, kBN, false, false);  // Q, K both K-major
-      constexpr uint32_t kIdO = idesc_bf16(kBM, D, false, true);     // P from TMEM, V MN-major
+      constexpr uint32_t kIdS = idesc_16(kBM, kBN, false, false, F16);  // Q, K both K-major
+      constexpr uint32_t kIdO = idesc_16(kBM, D, false, true, F16);    // P from TMEM, V MN-major
       auto issue_s = [&](int t, int j) {
         const uint32_t qa = sb + L::kOffQ + t * L::kTile;
         const uint32_t kb = sb + L::kOffK + (j % L::kStages) * L::kTile;
@@ -290,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       __uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]));
         const float2 p = exp2_pair(__ffma2_rn(sv, sl2, neg2), poly_pair<D>(c));
         sum[c & 1] = __fadd2_rn(sum[c & 1], p);
-        pk[c >> 5][c & 31] = pack_bf16(p.x, p.y);
+        pk[c >> 5][c & 31] = pack16<F16>(p.x, p.y);
       }
       l = l * alpha + ((sum[0].x + sum[0].y) + (sum[1].x + sum[1].y));
       m = m_use;
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       raise_error(status, abort_flag, kStatusTimeout);
     } else if (nkv[t] > 0) {
       tc_fence_after();
-      // Epilogue: O / l -> bf16 into this warp's 32 rows of the (now idle) Q_t tile,
+      // Epilogue: O / l -> bf16 / fp16 into this warp's 32 rows of the (now idle) Q_t tile,
       // in the 128-byte-swizzled layout the O tensor map expects, then one TMA store
       // per warp (rows past N are clipped by the hardware).
       const float inv_l = 1.f / l;
@@ -340,10 +342,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q4 = 0; q4 < 4; ++q4) {
           const int chunk = (cc & 1) * 4 + q4;
           uint4 v;
-          v.x = pack_bf16(__uint_as_float(o[8 * q4 + 0]) * inv_l, __uint_as_float(o[8 * q4 + 1]) * inv_l);
-          v.y = pack_bf16(__uint_as_float(o[8 * q4 + 2]) * inv_l, __uint_as_float(o[8 * q4 + 3]) * inv_l);
-          v.z = pack_bf16(__uint_as_float(o[8 * q4 + 4]) * inv_l, __uint_as_float(o[8 * q4 + 5]) * inv_l);
-          v.w = pack_bf16(__uint_as_float(o[8 * q4 + 6]) * inv_l, __uint_as_float(o[8 * q4 + 7]) * inv_l);
+          v.x = pack16<F16>(__uint_as_float(o[8 * q4 + 0]) * inv_l, __uint_as_float(o[8 * q4 + 1]) * inv_l);
+          v.y = pack16<F16>(__uint_as_float(o[8 * q4 + 2]) * inv_l, __uint_as_float(o[8 * q4 + 3]) * inv_l);
+          v.z = pack16<F16>(__uint_as_float(o[8 * q4 + 4]) * inv_l, __uint_as_float(o[8 * q4 + 5]) * inv_l);
+          v.w = pack16<F16>(__uint_as_float(o[8 * q4 + 6]) * inv_l, __uint_as_float(o[8 * q4 + 7]) * inv_l);
           *reinterpret_cast<uint4*>(stage + box * L::kBox + r * 128 + ((chunk ^ (r & 7)) << 4)) = v;
         }
       }
@@ -368,10 +370,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F16>
 cudaError_t launch_impl(const FwdLaunch& a, cudaStream_t stream) {
   using L = FwdSmem<D>;
-  auto kern = fwd_bf16_kernel<D, CAUSAL>;
+  auto kern = fwd_kernel<D, CAUSAL, F16>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
   if (e != cudaSuccess) return e;
   const int nqb = (a.N + 2 * kBM - 1) / (2 * kBM);
@@ -382,11 +384,16 @@ cudaError_t launch_impl(const FwdLaunch& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+template <bool F16>
+cudaError_t launch_typed(const FwdLaunch& a, cudaStream_t stream) {
+  if (a.D == 64) return a.causal ? launch_impl<64, true, F16>(a, stream) : launch_impl<64, false, F16>(a, stream);
+  return a.causal ? launch_impl<128, true, F16>(a, stream) : launch_impl<128, false, F16>(a, stream);
+}
+
 }  // namespace
 
-cudaError_t launch_fwd_bf16(const FwdLaunch& a, cudaStream_t stream) {
-  if (a.D == 64) return a.causal ? launch_impl<64, true>(a, stream) : launch_impl<64, false>(a, stream);
-  return a.causal ? launch_impl<128, true>(a, stream) : launch_impl<128, false>(a, stream);
+cudaError_t launch_fwd_16(const FwdLaunch& a, cudaStream_t stream) {
+  return a.f16 ? launch_typed<true>(a, stream) : launch_typed<false>(a, stream);
 }
 
 }  // namespace fa

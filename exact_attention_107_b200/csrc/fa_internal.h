@@ -8,18 +8,19 @@ namespace fa {
 
 constexpr int kStatusTimeout = 7;  // FA_ERR_TIMEOUT
 
-// bf16 forward (fa_fwd_sm100.cu).  Tensor maps are 3-D (D, N, B*H) bf16 with
-// 64 x 128 x 1 boxes and 128-byte swizzle.
+// bf16 / fp16 forward (fa_fwd_sm100.cu).  Tensor maps are 3-D (D, N, B*H) of the
+// element type with 64 x 128 x 1 boxes (O: 64 x 32 x 1) and 128-byte swizzle.
 struct FwdLaunch {
   CUtensorMap tmQ, tmK, tmV, tmO;
   float* lse;
   int BH, N, D;
   float scale;
   int causal;
+  int f16;           // element type: 0 = bf16, 1 = fp16
   int* status;
   int num_sms;
 };
-cudaError_t launch_fwd_bf16(const FwdLaunch& a, cudaStream_t stream);
+cudaError_t launch_fwd_16(const FwdLaunch& a, cudaStream_t stream);
 
 // fp32 forward (fa_fwd_f32.cu), plain pointers.
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
@@ -39,6 +40,7 @@ struct BwdLaunch {
   int BH, N, Npad, D;
   float scale;
   int causal;
+  int f16;           // element type of q, k, v, o, dO and the gradients: 0 = bf16, 1 = fp16
   int* status;
   int num_sms;
 };

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 namespace fa {
 
@@ -207,14 +208,17 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   d |= (uint64_t)2 << 61;   // layout: 128-byte swizzle
   return d;
 }
-// Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulate, dense.
-// a_mn / b_mn select MN-major (transposed) operands.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+// Instruction descriptor, kind::f16 with bf16 (or, when f16, fp16) A and B and fp32
+// accumulate, dense.  a_mn / b_mn select MN-major (transposed) operands.
+__host__ __device__ constexpr uint32_t idesc_16(int M, int N, bool a_mn, bool b_mn, bool f16) {
   return (1u << 4)                      // D format: f32
-         | (1u << 7)                    // A format: bf16
-         | (1u << 10)                   // B format: bf16
+         | ((f16 ? 0u : 1u) << 7)       // A format: f16 (0) or bf16 (1)
+         | ((f16 ? 0u : 1u) << 10)      // B format: same type as A
          | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
+  return idesc_16(M, N, a_mn, b_mn, false);
 }
 
 // ----------------------------------------------------------------------------- math
@@ -256,6 +260,27 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+// Same for fp16x2.
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// 16-bit element type of the kernels: bf16 or (F16) fp16, packed two per 32-bit word.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack16(float lo, float hi) {
+  return F16 ? pack_f16(lo, hi) : pack_bf16(lo, hi);
+}
+template <bool F16>
+__device__ __forceinline__ float unpack16_lo(uint32_t x) {
+  if (F16) return __half2float(__ushort_as_half(static_cast<unsigned short>(x & 0xffffu)));
+  return __uint_as_float(x << 16);
+}
+template <bool F16>
+__device__ __forceinline__ float unpack16_hi(uint32_t x) {
+  if (F16) return __half2float(__ushort_as_half(static_cast<unsigned short>(x >> 16)));
+  return __uint_as_float(x & 0xffff0000u);
 }
 
 // Three-input maximum (one instruction on sm_100).

@@ -25,8 +25,8 @@
  *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *     stream).  Every call is asynchronous on that stream; the library does no
  *     host synchronisation.
- *   - Supported: B, H, N >= 1; D in {64, 128} for bf16; D in {32, 64, 128} for
- *     fp32; Nq == Nk == N; causal in {0, 1}; ceil(N/256)*B*H < 2^31 (and
+ *   - Supported: B, H, N >= 1; D in {64, 128} for bf16 and fp16; D in
+ *     {32, 64, 128} for fp32; Nq == Nk == N; causal in {0, 1}; ceil(N/256)*B*H < 2^31 (and
  *     B*H <= 65535 for fa_fwd_f32).
  *   - Return value: FA_OK (0) or an fa_status code.  Arguments are validated
  *     before anything is launched; on an error nothing is launched and no
@@ -68,6 +68,18 @@ typedef enum {
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            int B, int H, int N, int D, float scale, int causal, void* stream);
 
+/* Forward with fp16 (IEEE binary16) q, k, v and o instead of bf16; otherwise
+ * identical to fa_fwd (fp32 accumulation and softmax, fp32 lse).  FP16 is the
+ * element type in which "CUDA-kernel-level optimisation: why Flash Attention is
+ * 5-10x faster than native PyTorch" (guanweilu.cn, section "three lines of
+ * PyTorch") and "Flash Attention principles: making Transformers faster"
+ * (ijyty.com, section "memory bottleneck") size the N x N matrices.  P is
+ * rounded to fp16 for the P V product, so it carries 3 more mantissa bits than
+ * on the bf16 path.  Values of O beyond the fp16 range (|x| > 65504) become
+ * +-inf. */
+int fa_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse,
+               int B, int H, int N, int D, float scale, int causal, void* stream);
+
 /* Forward in fp32 throughout (fp32 in, fp32 FFMA arithmetic, fp32 out), for
  * callers that need ~1e-6 relative accuracy.  Same arguments as fa_fwd with
  * float32 tensors. */
@@ -95,6 +107,15 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o, const voi
            const float* lse, void* dq, void* dk, void* dv,
            void* workspace, size_t workspace_bytes,
            int B, int H, int N, int D, float scale, int causal, void* stream);
+
+/* Backward with fp16 q, k, v, o, dO, dq, dk, dv (o and lse from fa_fwd_f16);
+ * otherwise identical to fa_bwd, with the same workspace.  P and dS are rounded
+ * to fp16 for the tensor-core products; gradients beyond the fp16 range become
+ * +-inf. */
+int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o, const void* dO,
+               const float* lse, void* dq, void* dk, void* dv,
+               void* workspace, size_t workspace_bytes,
+               int B, int H, int N, int D, float scale, int causal, void* stream);
 
 /* Backward stage 1: fills the workspace (layout above) from O, dO and lse. */
 int fa_bwd_preprocess(const void* o, const void* dO, const float* lse,

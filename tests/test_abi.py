@@ -103,3 +103,30 @@ def test_binding_requires_cuda_tensors():
     q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         fa.fa_fwd(q, q, q, q, torch.zeros(1, 1, 128), 0.125, False)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(v=Z), 1), (dict(N=0), 2), (dict(D=96), 3), (dict(q=U), 4), (dict(scale=float("inf")), 10),
+])
+def test_fwd_f16_rejects_bad_arguments(kw, code):
+    a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=2, N=256, D=64, scale=0.125, causal=0)
+    a.update(kw)
+    assert fa.load_library().fa_fwd_f16(*a.values(), None) == code
+
+
+def test_bwd_f16_rejects_bad_arguments():
+    lib = fa.load_library()
+    ws = lib.fa_bwd_workspace_size(1, 2, 256, 64)
+    args = [P] * 9
+    assert lib.fa_bwd_f16(*args, Z, ws, 1, 2, 256, 64, 0.125, 0, None) == 8
+    assert lib.fa_bwd_f16(*args[:5], Z, *args[6:], P, ws, 1, 2, 256, 64, 0.125, 0, None) == 1
+    assert lib.fa_bwd_f16(*args[:6], U, *args[7:], P, ws, 1, 2, 256, 64, 0.125, 0, None) == 4
+    assert lib.fa_bwd_f16(*args, P, ws, 1, 2, 256, 32, 0.125, 0, None) == 3
+    assert lib.fa_bwd_f16(*args, P, ws, 1, 2, 256, 64, 0.125, 3, None) == 10
+
+
+def test_binding_checks_fp16_dtype():
+    import torch
+    q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):      # not on a CUDA device: rejected before the dtype
+        fa.fa_fwd_f16(q, q, q, q, torch.zeros(1, 1, 128), 0.125, False)

@@ -32,7 +32,7 @@ class Workload:
     N: int
     D: int
     causal: bool
-    dtype: str            # "bf16" or "fp32": the storage/input type
+    dtype: str            # "bf16", "fp16" or "fp32": the storage/input type
     backward: bool        # does the workload include the backward pass
     seed: int
     qkv_std: float = 1.0
@@ -45,7 +45,7 @@ class Workload:
 
     @property
     def torch_dtype(self) -> torch.dtype:
-        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+        return {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}[self.dtype]
 
     def fwd_flops(self) -> float:
         """Algorithmic forward FLOPs: 4*B*H*N^2*D, halved when causal."""
