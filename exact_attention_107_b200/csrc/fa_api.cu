@@ -67,9 +67,11 @@ int device_state(DeviceState** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int check_shape(int B, int H, int N, int D, bool bf16) {
+// Head dims: 32, 64, 96, 128 on the 16-bit paths (32 and 96 run the 64- and 128-column
+// kernels on zero-filled columns); 32, 64, 128 on the fp32 forward.
+int check_shape(int B, int H, int N, int D, bool sixteen_bit) {
   if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
-  if (bf16 ? (D != 64 && D != 128) : (D != 32 && D != 64 && D != 128)) return FA_ERR_HEADDIM;
+  if (D != 32 && D != 64 && D != 128 && !(sixteen_bit && D == 96)) return FA_ERR_HEADDIM;
   const long long bh = static_cast<long long>(B) * H;
   if (bh > INT_MAX / 2) return FA_ERR_SHAPE;
   // The largest grid (ceil(N/128) * B*H CTAs, the dK/dV kernel) must fit a 31-bit grid.

@@ -46,13 +46,14 @@ constexpr int kPolyPer8 = 2;
 __device__ __forceinline__ bool poly_pair(int c2) { return (c2 & 7) >= 8 - kPolyPer8; }
 
 // ----------------------------------------------------------------------------- stage 1
-template <int D, bool F16>
+// kLanesPerRow lanes per row (a power of two, 8 * kLanesPerRow >= D), each reading 8
+// values (16 bytes) of O and of dO; lanes past the row's D columns read nothing.
+template <int kLanesPerRow, bool F16>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint16_t* __restrict__ o,
                                                              const uint16_t* __restrict__ dO,
                                                              const float* __restrict__ lse,
                                                              float* __restrict__ ws_nl, float* __restrict__ ws_delta,
-                                                             int N, int Npad, long long padded_rows) {
-  constexpr int kLanesPerRow = D / 8;   // each lane reads 8 values (16 bytes) of O and of dO
+                                                             int N, int Npad, int D, long long padded_rows) {
   const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long prow = gt / kLanesPerRow;          // row in the padded (B*H, Npad) layout
   const int part = static_cast<int>(gt % kLanesPerRow);
@@ -61,7 +62,7 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint16_t* __r
   const bool real = prow < padded_rows && n < N;
   const long long row = bh * N + n;                  // row in the caller's (B*H, N) layout
   float acc = 0.f;
-  if (real) {
+  if (real && part * 8 < D) {
     const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
     const uint4 b = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
     const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
@@ -750,15 +751,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool F16>
+template <int kLanesPerRow, bool F16>
 cudaError_t preprocess_impl(const BwdLaunch& a, cudaStream_t stream) {
   const long long padded_rows = static_cast<long long>(a.BH) * a.Npad;
-  const long long threads = padded_rows * (D / 8);
+  const long long threads = padded_rows * kLanesPerRow;
   const long long blocks = (threads + 255) / 256;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  bwd_preprocess_kernel<D, F16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+  bwd_preprocess_kernel<kLanesPerRow, F16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
       static_cast<const uint16_t*>(a.o), static_cast<const uint16_t*>(a.dO), a.lse, a.ws_nl, a.ws_delta,
-      a.N, a.Npad, padded_rows);
+      a.N, a.Npad, a.D, padded_rows);
   return cudaGetLastError();
 }
 
@@ -788,18 +789,21 @@ cudaError_t dq_impl(const BwdLaunch& a, cudaStream_t stream) {
 
 template <bool F16>
 cudaError_t preprocess_typed(const BwdLaunch& a, cudaStream_t stream) {
-  return a.D == 64 ? preprocess_impl<64, F16>(a, stream) : preprocess_impl<128, F16>(a, stream);
+  if (a.D <= 32) return preprocess_impl<4, F16>(a, stream);
+  return a.D <= 64 ? preprocess_impl<8, F16>(a, stream) : preprocess_impl<16, F16>(a, stream);
 }
 
 template <bool F16>
 cudaError_t dkdv_typed(const BwdLaunch& a, cudaStream_t stream) {
-  if (a.D == 64) return a.causal ? dkdv_impl<64, true, F16>(a, stream) : dkdv_impl<64, false, F16>(a, stream);
+  // Head dims 32 and 96 run the 64- and 128-column kernels on zero-filled tile columns
+  // (the tensor maps describe the caller's D), as in the forward.
+  if (a.D <= 64) return a.causal ? dkdv_impl<64, true, F16>(a, stream) : dkdv_impl<64, false, F16>(a, stream);
   return a.causal ? dkdv_impl<128, true, F16>(a, stream) : dkdv_impl<128, false, F16>(a, stream);
 }
 
 template <bool F16>
 cudaError_t dq_typed(const BwdLaunch& a, cudaStream_t stream) {
-  if (a.D == 64) return a.causal ? dq_impl<64, true, F16>(a, stream) : dq_impl<64, false, F16>(a, stream);
+  if (a.D <= 64) return a.causal ? dq_impl<64, true, F16>(a, stream) : dq_impl<64, false, F16>(a, stream);
   return a.causal ? dq_impl<128, true, F16>(a, stream) : dq_impl<128, false, F16>(a, stream);
 }
 

@@ -386,7 +386,11 @@ cudaError_t launch_impl(const FwdLaunch& a, cudaStream_t stream) {
 
 template <bool F16>
 cudaError_t launch_typed(const FwdLaunch& a, cudaStream_t stream) {
-  if (a.D == 64) return a.causal ? launch_impl<64, true, F16>(a, stream) : launch_impl<64, false, F16>(a, stream);
+  // Head dims 32 and 96 run the 64- and 128-column kernels: the tensor maps describe
+  // the caller's D, so the TMA fills the missing columns of every loaded tile with
+  // zeros (which add nothing to Q K^T and give zero columns of P V) and clips them
+  // from every store.
+  if (a.D <= 64) return a.causal ? launch_impl<64, true, F16>(a, stream) : launch_impl<64, false, F16>(a, stream);
   return a.causal ? launch_impl<128, true, F16>(a, stream) : launch_impl<128, false, F16>(a, stream);
 }
 

@@ -40,7 +40,8 @@ def test_workspace_size():
     assert fa.fa_bwd_workspace_size(1, 8, 65536, 128) == 2 * 8 * 65536 * 4
     assert fa.fa_bwd_workspace_size(1, 1, 3, 64) == 2 * 128 * 4
     assert fa.fa_bwd_workspace_size(2, 3, 129, 64) == 2 * 6 * 256 * 4
-    assert fa.fa_bwd_workspace_size(1, 1, 128, 96) == 0          # unsupported D
+    assert fa.fa_bwd_workspace_size(1, 1, 128, 96) == 2 * 128 * 4
+    assert fa.fa_bwd_workspace_size(1, 1, 128, 80) == 0          # unsupported D
 
 
 def test_noalloc_capacity_check_needs_no_gpu():
@@ -63,7 +64,7 @@ def _fwd(q=P, k=P, v=P, o=P, lse=P, B=1, H=2, N=256, D=64, scale=0.125, causal=0
 @pytest.mark.parametrize("kw,code", [
     (dict(q=Z), 1), (dict(lse=Z), 1),
     (dict(B=0), 2), (dict(N=0), 2), (dict(H=-1), 2), (dict(B=2**30, H=2**30), 2),
-    (dict(D=96), 3), (dict(D=32), 3), (dict(D=256), 3),
+    (dict(D=48), 3), (dict(D=16), 3), (dict(D=256), 3), (dict(D=80), 3),
     (dict(k=U), 4), (dict(o=U), 4),
     (dict(scale=float("nan")), 10), (dict(scale=0.0), 10), (dict(scale=-1.0), 10), (dict(causal=2), 10),
 ])
@@ -75,6 +76,7 @@ def test_fwd_f32_rejects_bad_arguments():
     lib = fa.load_library()
     assert lib.fa_fwd_f32(Z, P, P, P, P, 1, 1, 64, 64, 0.1, 0, None) == 1
     assert lib.fa_fwd_f32(P, P, P, P, P, 1, 1, 64, 48, 0.1, 0, None) == 3
+    assert lib.fa_fwd_f32(P, P, P, P, P, 1, 1, 64, 96, 0.1, 0, None) == 3     # 96: 16-bit paths only
     assert lib.fa_fwd_f32(P, P, P, P, P, 300, 300, 64, 64, 0.1, 0, None) == 2   # B*H > 65535
 
 
@@ -106,7 +108,7 @@ def test_binding_requires_cuda_tensors():
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(v=Z), 1), (dict(N=0), 2), (dict(D=96), 3), (dict(q=U), 4), (dict(scale=float("inf")), 10),
+    (dict(v=Z), 1), (dict(N=0), 2), (dict(D=48), 3), (dict(q=U), 4), (dict(scale=float("inf")), 10),
 ])
 def test_fwd_f16_rejects_bad_arguments(kw, code):
     a = dict(q=P, k=P, v=P, o=P, lse=P, B=1, H=2, N=256, D=64, scale=0.125, causal=0)
@@ -121,7 +123,7 @@ def test_bwd_f16_rejects_bad_arguments():
     assert lib.fa_bwd_f16(*args, Z, ws, 1, 2, 256, 64, 0.125, 0, None) == 8
     assert lib.fa_bwd_f16(*args[:5], Z, *args[6:], P, ws, 1, 2, 256, 64, 0.125, 0, None) == 1
     assert lib.fa_bwd_f16(*args[:6], U, *args[7:], P, ws, 1, 2, 256, 64, 0.125, 0, None) == 4
-    assert lib.fa_bwd_f16(*args, P, ws, 1, 2, 256, 32, 0.125, 0, None) == 3
+    assert lib.fa_bwd_f16(*args, P, ws, 1, 2, 256, 112, 0.125, 0, None) == 3
     assert lib.fa_bwd_f16(*args, P, ws, 1, 2, 256, 64, 0.125, 3, None) == 10
 
 

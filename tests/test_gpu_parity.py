@@ -53,6 +53,20 @@ def test_backward_small(B, H, N, D, causal):
     check_grads(got, ref, (B, H, N, D, causal))
 
 
+# Head dims 32 and 96 run the 64- and 128-column kernels on zero-filled columns.
+ODD_D = [(1, 2, 256, 32, False), (1, 2, 200, 32, True), (2, 1, 640, 32, True),
+         (1, 2, 256, 96, True), (2, 2, 333, 96, False), (1, 1, 1, 96, True)]
+
+
+@pytest.mark.parametrize("B,H,N,D,causal", ODD_D)
+def test_head_dims_32_and_96(B, H, N, D, causal):
+    w, (q, k, v, do) = _small(B, H, N, D, causal)
+    got = gpu_fwd_bwd(q, k, v, do, w.softmax_scale, causal)
+    ref = oracle.attention_backward(q, k, v, do, w.softmax_scale, causal)
+    check_fwd(got["O"], got["lse"], ref["O"], ref["lse"], (B, H, N, D, causal))
+    check_grads(got, ref, (B, H, N, D, causal))
+
+
 @pytest.mark.parametrize("D,causal", [(64, False), (128, True)])
 def test_large_logits_and_growing_max(D, causal):
     """Scores of large magnitude whose row max keeps growing along the keys, so the
