@@ -68,10 +68,12 @@ int device_state(DeviceState** out) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Head dims: 32, 64, 96, 128 on the 16-bit paths (32 and 96 run the 64- and 128-column
-// kernels on zero-filled columns); 32, 64, 128 on the fp32 forward.
-int check_shape(int B, int H, int N, int D, bool sixteen_bit) {
+// kernels on zero-filled columns) and 256 on the 16-bit forward (with_256); 32, 64, 128
+// on the fp32 forward.
+int check_shape(int B, int H, int N, int D, bool sixteen_bit, bool with_256 = false) {
   if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
-  if (D != 32 && D != 64 && D != 128 && !(sixteen_bit && D == 96)) return FA_ERR_HEADDIM;
+  if (D != 32 && D != 64 && D != 128 && !(sixteen_bit && D == 96) && !(with_256 && D == 256))
+    return FA_ERR_HEADDIM;
   const long long bh = static_cast<long long>(B) * H;
   if (bh > INT_MAX / 2) return FA_ERR_SHAPE;
   // The largest grid (ceil(N/128) * B*H CTAs, the dK/dV kernel) must fit a 31-bit grid.
@@ -141,7 +143,7 @@ int fa_device_status(int reset) {
 static int fwd16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int D,
                  float scale, int causal, void* stream, bool f16) {
   if (!q || !k || !v || !o || !lse) return FA_ERR_NULL;
-  int st = check_shape(B, H, N, D, true);
+  int st = check_shape(B, H, N, D, true, true);
   if (st != FA_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
   if (!scale_ok(scale) || (causal != 0 && causal != 1)) return FA_ERR_ARG;
@@ -162,7 +164,8 @@ static int fwd16(const void* q, const void* k, const void* v, void* o, float* ls
   a.causal = causal;
   a.status = ds->status;
   a.num_sms = ds->num_sms;
-  return launch_status(fa::launch_fwd_16(a, static_cast<cudaStream_t>(stream)));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return launch_status(D == 256 ? fa::launch_fwd_d256(a, s) : fa::launch_fwd_16(a, s));
 }
 
 extern "C" {

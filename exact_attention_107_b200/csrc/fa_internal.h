@@ -21,6 +21,8 @@ struct FwdLaunch {
   int num_sms;
 };
 cudaError_t launch_fwd_16(const FwdLaunch& a, cudaStream_t stream);
+// Head dimension 256 (fa_fwd_d256_sm100.cu): one query tile per CTA, same tensor maps.
+cudaError_t launch_fwd_d256(const FwdLaunch& a, cudaStream_t stream);
 
 // fp32 forward (fa_fwd_f32.cu), plain pointers.
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,

@@ -42,6 +42,7 @@ def test_workspace_size():
     assert fa.fa_bwd_workspace_size(2, 3, 129, 64) == 2 * 6 * 256 * 4
     assert fa.fa_bwd_workspace_size(1, 1, 128, 96) == 2 * 128 * 4
     assert fa.fa_bwd_workspace_size(1, 1, 128, 80) == 0          # unsupported D
+    assert fa.fa_bwd_workspace_size(1, 1, 128, 256) == 0         # D = 256: forward only
 
 
 def test_noalloc_capacity_check_needs_no_gpu():
@@ -64,7 +65,7 @@ def _fwd(q=P, k=P, v=P, o=P, lse=P, B=1, H=2, N=256, D=64, scale=0.125, causal=0
 @pytest.mark.parametrize("kw,code", [
     (dict(q=Z), 1), (dict(lse=Z), 1),
     (dict(B=0), 2), (dict(N=0), 2), (dict(H=-1), 2), (dict(B=2**30, H=2**30), 2),
-    (dict(D=48), 3), (dict(D=16), 3), (dict(D=256), 3), (dict(D=80), 3),
+    (dict(D=48), 3), (dict(D=16), 3), (dict(D=512), 3), (dict(D=80), 3), (dict(D=192), 3),
     (dict(k=U), 4), (dict(o=U), 4),
     (dict(scale=float("nan")), 10), (dict(scale=0.0), 10), (dict(scale=-1.0), 10), (dict(causal=2), 10),
 ])
@@ -90,6 +91,7 @@ def test_bwd_rejects_bad_arguments():
     assert lib.fa_bwd(*args[:8], U, P, ws, 1, 2, 256, 64, 0.125, 0, None) == 4
     assert lib.fa_bwd(*args[:3], Z, *args[4:], P, ws, 1, 2, 256, 64, 0.125, 0, None) == 1
     assert lib.fa_bwd(*args, P, ws, 1, 2, 256, 80, 0.125, 0, None) == 3
+    assert lib.fa_bwd(*args, P, ws, 1, 2, 256, 256, 0.125, 0, None) == 3     # D = 256: forward only
     ws1 = lib.fa_bwd_workspace_size(1, 1, 128, 64)
     assert ws1 == 2 * 128 * 4
     assert lib.fa_bwd_dq(P, P, P, P, P, ws1, Z, 1, 1, 128, 64, 0.1, 0, None) == 1

@@ -20,6 +20,16 @@ SHAPES = [
 ]
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp16_forward_head_dim_256(causal):
+    w, (q, k, v, do) = _inputs(1, 2, 640, 256, causal)
+    O, lse = fa.attention_forward(q.cuda(), k.cuda(), v.cuda(), w.softmax_scale, causal)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status(reset=True) == 0
+    ref_O, ref_lse = oracle.attention_forward(q, k, v, w.softmax_scale, causal)
+    check_fwd(O.cpu(), lse.cpu(), ref_O, ref_lse, tol=TOL_F16)
+
+
 @pytest.fixture(autouse=True)
 def _need_cuda(cuda_ok):
     yield

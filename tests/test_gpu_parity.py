@@ -67,6 +67,39 @@ def test_head_dims_32_and_96(B, H, N, D, causal):
     check_grads(got, ref, (B, H, N, D, causal))
 
 
+# Head dim 256: forward only (its own kernel: one query tile per CTA, two score buffers).
+D256 = [(1, 2, 256, 256, False), (1, 2, 384, 256, True), (2, 1, 200, 256, True), (1, 1, 1, 256, False),
+        (1, 3, 1000, 256, False), (1, 2, 1024, 256, True)]
+
+
+@pytest.mark.parametrize("B,H,N,D,causal", D256)
+def test_forward_head_dim_256(B, H, N, D, causal):
+    w, (q, k, v, do) = _small(B, H, N, D, causal)
+    O, lse, _ = gpu_forward(q, k, v, w.softmax_scale, causal)
+    ref_O, ref_lse = oracle.attention_forward(q, k, v, w.softmax_scale, causal)
+    check_fwd(O.cpu(), lse.cpu(), ref_O, ref_lse, (B, H, N, D, causal))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_forward_head_dim_256_growing_max(causal):
+    """The rescale of the 256-column accumulator, which waits for the previous P V product."""
+    B, H, N, D = 1, 2, 1024, 256
+    w, (q, k, v, do) = _small(B, H, N, D, causal, seed=5)
+    ramp = torch.linspace(0.2, 3.0, N).view(1, 1, N, 1)
+    k = (k.float() * ramp).to(torch.bfloat16)
+    q = (q.float() * 2.0).to(torch.bfloat16)
+    O, lse, _ = gpu_forward(q, k, v, w.softmax_scale, causal)
+    ref_O, ref_lse = oracle.attention_forward(q, k, v, w.softmax_scale, causal)
+    check_fwd(O.cpu(), lse.cpu(), ref_O, ref_lse)
+
+
+def test_backward_head_dim_256_is_rejected():
+    q = torch.zeros(1, 1, 128, 256, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(1, 1, 128, device="cuda")
+    with pytest.raises(fa.FAError):
+        fa.attention_backward(q, q, q, q, lse, q, 0.0625, False)
+
+
 @pytest.mark.parametrize("D,causal", [(64, False), (128, True)])
 def test_large_logits_and_growing_max(D, causal):
     """Scores of large magnitude whose row max keeps growing along the keys, so the
