@@ -2,6 +2,7 @@
 
     python bench_sweep.py nsweep   [--H 8] [--D 128] [--causal 1] [--Ns 1024,2048,...] [--dtype fp16]
     python bench_sweep.py standard [--workload c3_bf16_fwdbwd]
+    python bench_sweep.py fwd      [--B 1] [--H 16] [--N 16384] [--D 256] [--causal 1] [--dtype bf16]
 
 nsweep: for each N, forward and backward time (CUDA events, median of 5 after 2
 warm-up runs) and peak device memory of the fused path (fa_fwd + fa_bwd through
@@ -13,6 +14,9 @@ PyTorch", guanweilu.cn).  The standard path is skipped where its N x N tensors
 would need more than --std-limit-gb of device memory.  Prints a markdown table.
 
 standard: the same comparison on one named workload, printing one JSON line.
+
+fwd: forward only (any supported head dim, 256 included), one JSON line with the median
+time of 10 launches after 3 warm-up launches and the attention TFLOP/s.
 
 Inputs are seeded N(0,1) draws rounded to bf16, or to fp16 with --dtype fp16 (the
 recipe of workloads.py).
@@ -140,20 +144,29 @@ def standard(args):
                       "speedup": {"fwd": sf / ff, "bwd": sb / fb, "fwd_bwd": (sf + sb) / (ff + fb)}}))
 
 
+def fwd_only(args):
+    w, (q, k, v, do) = inputs(args.B, args.H, args.N, args.D, bool(args.causal), dtype=args.dtype)
+    fwd, _ = fused_step(q, k, v, do, w.softmax_scale, w.causal)
+    t = _time(fwd, warmup=3, reps=10)
+    assert fa.fa_device_status(reset=True) == 0
+    print(json.dumps({"workload": w.describe(), "fwd_ms": t, "fwd_tflops": w.fwd_flops() / t / 1e9}))
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("mode", choices=["nsweep", "standard"])
+    ap.add_argument("mode", choices=["nsweep", "standard", "fwd"])
     ap.add_argument("--B", type=int, default=1)
     ap.add_argument("--H", type=int, default=8)
     ap.add_argument("--D", type=int, default=128)
     ap.add_argument("--causal", type=int, default=1)
     ap.add_argument("--Ns", default="1024,2048,4096,8192,16384,32768,65536,131072")
+    ap.add_argument("--N", type=int, default=16384)
     ap.add_argument("--std-limit-gb", type=float, default=80.0)
     ap.add_argument("--dtype", choices=["bf16", "fp16"], default="bf16")
     ap.add_argument("--workload", default="c3_bf16_fwdbwd")
     args = ap.parse_args()
     torch.cuda.set_device(0)
-    nsweep(args) if args.mode == "nsweep" else standard(args)
+    {"nsweep": nsweep, "standard": standard, "fwd": fwd_only}[args.mode](args)
 
 
 if __name__ == "__main__":

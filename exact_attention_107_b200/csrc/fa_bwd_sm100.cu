@@ -310,9 +310,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + dcol, tmem + packed_col(abase, kk), mnmajor_desc(b_tile, kk, T::kBox), kIdAcc,
                  (!first || kk > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(bar(L::kBarKV), 0, abort_flag);
+      bool ok = mbar_wait_spin(bar(L::kBarKV), 0, abort_flag);
       if (ok && n > 0) {
-        ok = mbar_wait(bar(L::kBarQFull), 0, abort_flag) && mbar_wait(bar(L::kBarOFull), 0, abort_flag);
+        ok = mbar_wait_spin(bar(L::kBarQFull), 0, abort_flag) && mbar_wait_spin(bar(L::kBarOFull), 0, abort_flag);
         if (ok) {
           tc_fence_after();
           issue_st(0);
@@ -321,23 +321,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int i = 0; ok && i < n; ++i) {
         const int s = i % L::kStages;
-        if (!(ok = mbar_wait(bar(L::kBarP), i & 1, abort_flag))) break;
+        if (!(ok = mbar_wait_spin(bar(L::kBarP), i & 1, abort_flag))) break;
         tc_fence_after();
         issue_acc(kColDV, kColS, sb + L::kOffdO + s * T::kBytes, i == 0);        // dV += P^T dO_i
         tc_commit(bar(L::kBarOEmpty + s));
         if (i + 1 < n) {
           const int sn = (i + 1) % L::kStages;
-          if (!(ok = mbar_wait(bar(L::kBarQFull + sn), ((i + 1) / L::kStages) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait_spin(bar(L::kBarQFull + sn), ((i + 1) / L::kStages) & 1, abort_flag))) break;
           tc_fence_after();
           issue_st(i + 1);                                                       // over P^T_i (read above)
         }
-        if (!(ok = mbar_wait(bar(L::kBarDS), i & 1, abort_flag))) break;
+        if (!(ok = mbar_wait_spin(bar(L::kBarDS), i & 1, abort_flag))) break;
         tc_fence_after();
         issue_acc(kColDK, kColDP, sb + L::kOffQ + s * T::kBytes, i == 0);        // dK += dS^T Q_i
         tc_commit(bar(L::kBarQEmpty + s));
         if (i + 1 < n) {
           const int sn = (i + 1) % L::kStages;
-          if (!(ok = mbar_wait(bar(L::kBarOFull + sn), ((i + 1) / L::kStages) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait_spin(bar(L::kBarOFull + sn), ((i + 1) / L::kStages) & 1, abort_flag))) break;
           tc_fence_after();
           issue_dpt(i + 1);                                                      // over dS^T_i (read above)
         }
@@ -584,6 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait_drain(bar(L::kBarVFull + j % L::kVStages), (j / L::kVStages) & 1);
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_16(128, 128, false, false, F16);
       constexpr uint32_t kIdAcc = idesc_16(128, D, false, true, F16);
@@ -596,9 +597,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ss(tmem + 128 * t, kmajor_desc(sQ, kk, T::kBox), kmajor_desc(sK, kk, T::kBox), kIdS, kk > 0);
         tc_commit(bar(L::kBarS + t));
       };
-      bool ok = mbar_wait(bar(L::kBarQ), 0, abort_flag);
+      bool ok = mbar_wait_spin(bar(L::kBarQ), 0, abort_flag);
       if (ok && nmax > 0) {
-        ok = mbar_wait(bar(L::kBarKFull), 0, abort_flag);
+        ok = mbar_wait_spin(bar(L::kBarKFull), 0, abort_flag);
         if (ok) {
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
@@ -612,9 +613,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool v_ready = false;
         for (int t = 0; t < 2 && ok; ++t) {     // dP_t = dO_t V_j^T, over S_t once it has been read
           if (j >= nk[t]) continue;
-          if (!(ok = mbar_wait(bar(L::kBarSC + t), j & 1, abort_flag))) break;
+          if (!(ok = mbar_wait_spin(bar(L::kBarSC + t), j & 1, abort_flag))) break;
           if (!v_ready) {
-            if (!(ok = mbar_wait(bar(L::kBarVFull + vs), (j / L::kVStages) & 1, abort_flag))) break;
+            if (!(ok = mbar_wait_spin(bar(L::kBarVFull + vs), (j / L::kVStages) & 1, abort_flag))) break;
             v_ready = true;
           }
           tc_fence_after();
@@ -629,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool k_next = false;
         for (int t = 0; t < 2 && ok; ++t) {     // dQ_t += dS_t K_j, then S_t for the next key tile
           if (j >= nk[t]) continue;
-          if (!(ok = mbar_wait(bar(L::kBarDS + t), j & 1, abort_flag))) break;
+          if (!(ok = mbar_wait_spin(bar(L::kBarDS + t), j & 1, abort_flag))) break;
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 128 / 16; ++kk)    // dQ += dS K_j; dS half h packed at 64h + [0, 32)
@@ -639,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (j + 1 < nk[t]) {
             if (!k_next) {
               const int jn = j + 1;
-              if (!(ok = mbar_wait(bar(L::kBarKFull + jn % L::kKStages), (jn / L::kKStages) & 1, abort_flag)))
+              if (!(ok = mbar_wait_spin(bar(L::kBarKFull + jn % L::kKStages), (jn / L::kKStages) & 1, abort_flag)))
                 break;
               tc_fence_after();
               k_next = true;

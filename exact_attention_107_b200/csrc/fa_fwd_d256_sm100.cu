@@ -151,13 +151,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_16(kBM, kBN, false, false, F16);   // Q, K both K-major
-      constexpr uint32_t kIdO = idesc_16(kBM, 128, false, true, F16);    // P from TMEM, V MN-major, N = 128
+      constexpr uint32_t kIdO = idesc_16(kBM, kD, false, true, F16);     // P from TMEM, V MN-major, N = 256
       // S_j = Q K_j^T into buffer j & 1; each K box is released once its 4 K-steps finish.
       auto issue_s = [&](int j) -> bool {
         const int b0 = 4 * seq_k(j);
         for (int c = 0; c < L::kNBox; ++c) {
           const int b = b0 + c;
-          if (!mbar_wait(bar(L::kBarFull + (b & (L::kRing - 1))), (b >> 3) & 1, abort_flag)) return false;
+          if (!mbar_wait_spin(bar(L::kBarFull + (b & (L::kRing - 1))), (b >> 3) & 1, abort_flag)) return false;
           tc_fence_after();
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4)
@@ -168,30 +168,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(bar(L::kBarSFull + (j & 1)));
         return true;
       };
-      // O += P_j V_j as two N = 128 halves (V boxes 0-1, then 2-3).
+      // O += P_j V_j, one N = 256 MMA per 16 keys (an N = 256 MMA runs at the full rate,
+      // two N = 128 halves would not); the 4 V boxes are consecutive ring slots.
       auto issue_pv = [&](int j) -> bool {
-        if (!mbar_wait(bar(L::kBarPFull + (j & 1)), (j >> 1) & 1, abort_flag)) return false;
+        if (!mbar_wait_spin(bar(L::kBarPFull + (j & 1)), (j >> 1) & 1, abort_flag)) return false;
         const int b0 = 4 * seq_v(j, n);
         for (int c = 0; c < L::kNBox; ++c) {
           const int b = b0 + c;
-          if (!mbar_wait(bar(L::kBarFull + (b & (L::kRing - 1))), (b >> 3) & 1, abort_flag)) return false;
+          if (!mbar_wait_spin(bar(L::kBarFull + (b & (L::kRing - 1))), (b >> 3) & 1, abort_flag)) return false;
         }
         tc_fence_after();
+        const uint32_t vb = box(b0);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t vb = box(b0 + 2 * h);
-#pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            mma_ts(tmem + 256 + h * 128, tmem + (j & 1) * 128 + kk * 8, sdesc_sw128(vb + kk * 2048, L::kBox, 1024),
-                   kIdO, (j > 0 || kk > 0) ? 1u : 0u);
-          tc_commit(bar(L::kBarEmpty + ((b0 + 2 * h) & (L::kRing - 1))));
-          tc_commit(bar(L::kBarEmpty + ((b0 + 2 * h + 1) & (L::kRing - 1))));
-        }
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_ts(tmem + 256, tmem + (j & 1) * 128 + kk * 8, sdesc_sw128(vb + kk * 2048, L::kBox, 1024), kIdO,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        for (int c = 0; c < L::kNBox; ++c) tc_commit(bar(L::kBarEmpty + ((b0 + c) & (L::kRing - 1))));
         tc_commit(bar(L::kBarODone));
         if (j == n - 1) tc_commit(bar(L::kBarOFull));
         return true;
       };
-      bool ok = mbar_wait(bar(L::kBarQFull), 0, abort_flag);
+      bool ok = mbar_wait_spin(bar(L::kBarQFull), 0, abort_flag);
       if (ok) {
         tc_fence_after();
         ok = issue_s(0);

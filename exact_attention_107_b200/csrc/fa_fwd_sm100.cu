@@ -198,9 +198,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, sdesc_sw128(vb + kk * 2048, L::kBox, 1024), kIdO,
                  (j > 0 || kk > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(bar(L::kBarQFull), 0, abort_flag);
+      bool ok = mbar_wait_spin(bar(L::kBarQFull), 0, abort_flag);
       if (ok && nkv_max > 0) {
-        ok = mbar_wait(bar(L::kBarKFull), 0, abort_flag);
+        ok = mbar_wait_spin(bar(L::kBarKFull), 0, abort_flag);
         if (ok) {
           tc_fence_after();
           for (int t = 0; t < 2; ++t)
@@ -210,19 +210,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int j = 0; ok && j < nkv_max; ++j) {
         const int s = j % L::kStages;
-        if (!(ok = mbar_wait(bar(L::kBarVFull + s), (j / L::kStages) & 1, abort_flag))) break;
+        if (!(ok = mbar_wait_spin(bar(L::kBarVFull + s), (j / L::kStages) & 1, abort_flag))) break;
         tc_fence_after();
         bool k_next = false;
         for (int t = 0; t < 2; ++t) {
           if (j >= nkv[t]) continue;
-          if (!(ok = mbar_wait(bar(L::kBarPFull + t), j & 1, abort_flag))) break;
+          if (!(ok = mbar_wait_spin(bar(L::kBarPFull + t), j & 1, abort_flag))) break;
           tc_fence_after();
           issue_pv(t, j);
           if (j == nkv[t] - 1) tc_commit(bar(L::kBarOFull + t));
           if (j + 1 < nkv[t]) {
             if (!k_next) {
               const int jn = j + 1;
-              if (!(ok = mbar_wait(bar(L::kBarKFull + jn % L::kStages), (jn / L::kStages) & 1, abort_flag)))
+              if (!(ok = mbar_wait_spin(bar(L::kBarKFull + jn % L::kStages), (jn / L::kStages) & 1, abort_flag)))
                 break;
               tc_fence_after();
               k_next = true;
