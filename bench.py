@@ -237,21 +237,24 @@ def run_ours(args, rank, world, local_rank):
     # ---------------------------------------------------------------- end-to-end from host buffers
     e2e = None
     if not args.no_e2e:
+        # Every step uploads its inputs from pinned host memory and downloads O, lse, dQ,
+        # dK, dV; HostStepPipeline overlaps step i's kernels with the copies of its
+        # neighbours (two device buffer sets, separate copy streams).
         pinned = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
-        dev_bufs = {"q": q, "k": k, "v": v, "do": do, "o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv,
-                    "ws": ws}
-        out = {n: torch.empty(B, H, N, D, dtype=torch.bfloat16).pin_memory() for n in ("o", "dq", "dk", "dv")}
-        out["lse"] = torch.empty(B, H, N, dtype=torch.float32).pin_memory()
-        for _ in range(max(1, args.warmup)):
-            fa.attention_fwd_bwd_from_host(*pinned, scale, causal, dev_bufs, out, stream)
+        pipe = fa.HostStepPipeline(B, H, N, D, dtype=q.dtype, device=dev)
+        outs = [pipe.host_outputs() for _ in range(pipe.depth)]
+        for i in range(max(1, args.warmup)):
+            pipe.submit(*pinned, outs[i % pipe.depth], scale, causal)
+        pipe.synchronize()
         torch.cuda.synchronize(dev)
         if world > 1:
             torch.distributed.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            _, h2d, d2h = fa.attention_fwd_bwd_from_host(*pinned, scale, causal, dev_bufs, out, stream)
-        e1.record(stream)
+        e0.record(pipe.s_h2d)
+        for i in range(args.steps):
+            h2d, d2h = pipe.submit(*pinned, outs[i % pipe.depth], scale, causal)
+        e1.record(pipe.s_d2h)
+        pipe.synchronize()
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
         e2e = {"ms_per_step": e2e_ms / args.steps, "h2d": h2d, "d2h": d2h}

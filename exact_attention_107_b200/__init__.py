@@ -10,6 +10,7 @@ from ._binding import (  # noqa: F401
     SYMBOLS,
     FAError,
     FlashAttention,
+    HostStepPipeline,
     attention_backward,
     attention_forward,
     attention_fwd_bwd_from_host,

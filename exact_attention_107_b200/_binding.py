@@ -298,3 +298,74 @@ def attention_fwd_bwd_from_host(q_h, k_h, v_h, do_h, scale: float, causal: bool,
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, do_h))
     d2h = sum(t.numel() * t.element_size() for t in out.values())
     return out, h2d, d2h
+
+
+class HostStepPipeline:
+    """Forward + backward steps whose inputs and results live in pinned host memory,
+    pipelined over `depth` sets of device buffers and three CUDA streams: the upload of
+    step i+1 and the download of step i-1 run on the copy engines while step i computes.
+
+    submit(q, k, v, do, out, scale, causal) queues one step: copy q, k, v, dO (pinned
+    host tensors of shape (B,H,N,D)) to the device, fa_fwd + fa_bwd (or the fp16 entry
+    points) on the compute stream, then copy O, lse, dQ, dK, dV into `out` (a dict of
+    pinned host tensors, as returned by host_outputs()).  Results of a step are in `out`
+    once wait() (or synchronize()) has returned; a caller keeping several steps in flight
+    gives each its own `out`.  The library's own kernels do all the arithmetic; this class
+    only orders copies and launches."""
+
+    def __init__(self, B: int, H: int, N: int, D: int, dtype=torch.bfloat16, depth: int = 2, device=None):
+        dev = torch.device("cuda") if device is None else torch.device(device)
+        self.shape, self.dtype, self.depth = (B, H, N, D), dtype, depth
+        self.bufs = []
+        for _ in range(depth):
+            b = {n: torch.empty(B, H, N, D, device=dev, dtype=dtype)
+                 for n in ("q", "k", "v", "do", "o", "dq", "dk", "dv")}
+            b["lse"] = torch.empty(B, H, N, device=dev, dtype=torch.float32)
+            self.bufs.append(b)
+        self.ws = torch.empty(fa_bwd_workspace_size(B, H, N, D), device=dev, dtype=torch.uint8)
+        self.s_h2d, self.s_comp, self.s_d2h = (torch.cuda.Stream(dev) for _ in range(3))
+        self.ev_loaded = [torch.cuda.Event() for _ in range(depth)]    # inputs of the slot on the device
+        self.ev_computed = [torch.cuda.Event() for _ in range(depth)]  # slot's kernels done
+        self.ev_fetched = [torch.cuda.Event() for _ in range(depth)]   # slot's results copied out
+        self.used = [False] * depth
+        self.i = 0
+
+    def host_outputs(self):
+        B, H, N, D = self.shape
+        out = {n: torch.empty(B, H, N, D, dtype=self.dtype).pin_memory() for n in ("o", "dq", "dk", "dv")}
+        out["lse"] = torch.empty(B, H, N, dtype=torch.float32).pin_memory()
+        return out
+
+    def submit(self, q_h, k_h, v_h, do_h, out, scale: float, causal: bool):
+        """Queues one step; returns (h2d_bytes, d2h_bytes) of its copies."""
+        s = self.i % self.depth
+        b = self.bufs[s]
+        if self.used[s]:
+            self.s_h2d.wait_event(self.ev_computed[s])     # the kernels of step i-depth read these inputs
+        with torch.cuda.stream(self.s_h2d):
+            for n, h in (("q", q_h), ("k", k_h), ("v", v_h), ("do", do_h)):
+                b[n].copy_(h, non_blocking=True)
+        self.ev_loaded[s].record(self.s_h2d)
+        self.s_comp.wait_event(self.ev_loaded[s])
+        if self.used[s]:
+            self.s_comp.wait_event(self.ev_fetched[s])     # step i-depth's results have left these buffers
+        fwd, bwd = (fa_fwd_f16, fa_bwd_f16) if self.dtype == torch.float16 else (fa_fwd, fa_bwd)
+        fwd(b["q"], b["k"], b["v"], b["o"], b["lse"], scale, causal, self.s_comp)
+        bwd(b["q"], b["k"], b["v"], b["o"], b["do"], b["lse"], b["dq"], b["dk"], b["dv"], self.ws, scale, causal,
+            self.s_comp)
+        self.ev_computed[s].record(self.s_comp)
+        self.s_d2h.wait_event(self.ev_computed[s])
+        with torch.cuda.stream(self.s_d2h):
+            for n in ("o", "lse", "dq", "dk", "dv"):
+                out[n].copy_(b[n], non_blocking=True)
+        self.ev_fetched[s].record(self.s_d2h)
+        self.used[s] = True
+        self.i += 1
+        h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, do_h))
+        d2h = sum(out[n].numel() * out[n].element_size() for n in ("o", "lse", "dq", "dk", "dv"))
+        return h2d, d2h
+
+    def synchronize(self):
+        """Waits until every queued step's results are in host memory."""
+        for st in (self.s_h2d, self.s_comp, self.s_d2h):
+            st.synchronize()

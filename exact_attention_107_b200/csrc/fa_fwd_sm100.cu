@@ -22,7 +22,9 @@
 // O_1 [256+D, 256+2D).  P_t (16-bit, two per 32-bit column) overwrites the first 64
 // columns of S_t once the scores have been read into registers.  P_t takes the
 // element type of the inputs (bf16, or fp16 when F16), as the tensor-core operands
-// of one MMA share one type.
+// of one MMA share one type.  It is written and announced in two halves of 64 keys,
+// and the MMA thread issues the first half's P V products while the softmax computes
+// the second half.
 //
 // Online-softmax detail: the running max used for the exponentials is only raised
 // when a new row max exceeds it by more than 2^8 (in exp2 units).  Numerator and
@@ -65,8 +67,8 @@ struct FwdSmem {
   static constexpr int kBarVFull = kBarKEmpty + kStages;
   static constexpr int kBarVEmpty = kBarVFull + kStages;
   static constexpr int kBarSFull = kBarVEmpty + kStages;  // [2]
-  static constexpr int kBarPFull = kBarSFull + 2;         // [2]
-  static constexpr int kBarOFull = kBarPFull + 2;         // [2]
+  static constexpr int kBarPFull = kBarSFull + 2;         // [half][tile]: P of keys [64h, 64h+64)
+  static constexpr int kBarOFull = kBarPFull + 4;         // [2]
   static constexpr int kBarMmaDone = kBarOFull + 2;
   static constexpr int kNumBars = kBarMmaDone + 1;
   static constexpr int kOffSlot = kOffBar + 8 * kNumBars;  // TMEM base address, then abort flag
@@ -121,6 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(L::kBarSFull + t), 1);
       mbar_init(bar(L::kBarPFull + t), kBM);
+      mbar_init(bar(L::kBarPFull + 2 + t), kBM);
       mbar_init(bar(L::kBarOFull + t), 1);
     }
     mbar_init(bar(L::kBarMmaDone), 1);
@@ -191,10 +194,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit(bar(L::kBarSFull + t));
       };
-      auto issue_pv = [&](int t, int j) {
+      // O_t += P_t V_j over keys [64h, 64h+64): K-steps 4h .. 4h+3.
+      auto issue_pv = [&](int t, int j, int h) {
         const uint32_t vb = sb + L::kOffV + (j % L::kStages) * L::kTile;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
+        for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
           mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, sdesc_sw128(vb + kk * 2048, L::kBox, 1024), kIdO,
                  (j > 0 || kk > 0) ? 1u : 0u);
       };
@@ -215,9 +219,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool k_next = false;
         for (int t = 0; t < 2; ++t) {
           if (j >= nkv[t]) continue;
+          // P_t arrives in two halves; the first half's products start while the
+          // softmax still computes the second.
           if (!(ok = mbar_wait_spin(bar(L::kBarPFull + t), j & 1, abort_flag))) break;
           tc_fence_after();
-          issue_pv(t, j);
+          issue_pv(t, j, 0);
+          if (!(ok = mbar_wait_spin(bar(L::kBarPFull + 2 + t), j & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(t, j, 1);
           if (j == nkv[t] - 1) tc_commit(bar(L::kBarOFull + t));
           if (j + 1 < nkv[t]) {
             if (!k_next) {
@@ -283,43 +292,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_use = need ? m_new : m;
       const float alpha = need ? ex2_approx(m - m_new) : 1.f;
       const float neg = (m_use == -CUDART_INF_F) ? 0.f : -m_use;
-      uint32_t pk[2][32];
+      // P = exp2(s * scale * log2 e - m) in two halves of 64 keys; each half is stored as
+      // packed 16-bit pairs over the first 32 + 32 columns of S_t (already read) and
+      // announced on its own barrier, so the P V products of the first half overlap the
+      // exponentials of the second.
       float2 sum[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       const float2 sl2 = make_float2(scale_log2, scale_log2), neg2 = make_float2(neg, neg);
 #pragma unroll
-      for (int c = 0; c < kBN / 2; ++c) {
-        const float2 sv = make_float2(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]),
-                                      __uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]));
-        const float2 p = exp2_pair(__ffma2_rn(sv, sl2, neg2), poly_pair<D>(c));
-        sum[c & 1] = __fadd2_rn(sum[c & 1], p);
-        pk[c >> 5][c & 31] = pack16<F16>(p.x, p.y);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) {
+          const int c = 32 * h + c2;                       // pair index: columns 2c, 2c + 1
+          const float2 sv = make_float2(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]),
+                                        __uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]));
+          const float2 p = exp2_pair(__ffma2_rn(sv, sl2, neg2), poly_pair<D>(c));
+          sum[c & 1] = __fadd2_rn(sum[c & 1], p);
+          pk[c2] = pack16<F16>(p.x, p.y);
+        }
+        if (h == 0 && j > 0 && __any_sync(0xffffffffu, need)) {
+          // Rescale O_t before any of this step's P V products lands in it (after the
+          // first half's exponentials, whose scores no longer occupy registers).  O_t was
+          // finished by the PV MMAs of step j-1: the commit that announced S_t(j) also
+          // covers every earlier MMA of this thread, including those.
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_ld_wait();
+            reg_fence(o);
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
+                                          make_float2(alpha, alpha));
+              o[i] = __float_as_uint(v.x);
+              o[i + 1] = __float_as_uint(v.y);
+            }
+            tmem_st32(tO + cc * 32, o);
+          }
+        }
+        tmem_st32(tS + 32 * h, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::kBarPFull + 2 * h + t));
       }
       l = l * alpha + ((sum[0].x + sum[0].y) + (sum[1].x + sum[1].y));
       m = m_use;
-      tmem_st32(tS, pk[0]);
-      tmem_st32(tS + 32, pk[1]);
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // O_t was finished by the PV MMA of step j-1: the commit that announced S_t(j)
-        // also covers every earlier MMA of this thread, including that PV.
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tO + cc * 32, o);
-          tmem_ld_wait();
-          reg_fence(o);
-#pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            const float2 v = __fmul2_rn(make_float2(__uint_as_float(o[i]), __uint_as_float(o[i + 1])),
-                                        make_float2(alpha, alpha));
-            o[i] = __float_as_uint(v.x);
-            o[i + 1] = __float_as_uint(v.y);
-          }
-          tmem_st32(tO + cc * 32, o);
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(L::kBarPFull + t));
     }
     if (ok && nkv[t] > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarOFull + t), 0, abort_flag));
     if (!ok) {
