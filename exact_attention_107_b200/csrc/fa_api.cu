@@ -67,17 +67,17 @@ int device_state(DeviceState** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Head dims: 32, 64, 96, 128 on the 16-bit paths (32 and 96 run the 64- and 128-column
-// kernels on zero-filled columns) and 256 on the 16-bit forward (with_256); 32, 64, 128
-// on the fp32 forward.
+// Head dims: 32, 64, 96, 128 and (with_256) 256 on the 16-bit paths (32 and 96 run the
+// 64- and 128-column kernels on zero-filled columns); 32, 64, 128 on the fp32 forward.
 int check_shape(int B, int H, int N, int D, bool sixteen_bit, bool with_256 = false) {
   if (B < 1 || H < 1 || N < 1) return FA_ERR_SHAPE;
   if (D != 32 && D != 64 && D != 128 && !(sixteen_bit && D == 96) && !(with_256 && D == 256))
     return FA_ERR_HEADDIM;
   const long long bh = static_cast<long long>(B) * H;
   if (bh > INT_MAX / 2) return FA_ERR_SHAPE;
-  // The largest grid (ceil(N/128) * B*H CTAs, the dK/dV kernel) must fit a 31-bit grid.
-  if ((static_cast<long long>(N) + 127) / 128 * bh > INT_MAX) return FA_ERR_SHAPE;
+  // The largest grid (ceil(N/128) * B*H CTAs, the dK/dV kernel; twice that at D = 256)
+  // must fit a 31-bit grid.
+  if ((static_cast<long long>(N) + 127) / 128 * bh * (D == 256 ? 2 : 1) > INT_MAX) return FA_ERR_SHAPE;
   return FA_OK;
 }
 
@@ -195,7 +195,7 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int D) {
-  if (check_shape(B, H, N, D, true) != FA_OK) return 0;
+  if (check_shape(B, H, N, D, true, true) != FA_OK) return 0;
   const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
   return 2 * static_cast<size_t>(B) * H * npad * sizeof(float);    // a multiple of 1024 bytes
 }
@@ -215,7 +215,7 @@ static int workspace_views(void* ws, size_t ws_bytes, int B, int H, int N, int D
 static int preprocess16(const void* o, const void* dO, const float* lse, void* workspace, size_t workspace_bytes,
                         int B, int H, int N, int D, void* stream, bool f16) {
   if (!o || !dO || !lse) return FA_ERR_NULL;
-  int st = check_shape(B, H, N, D, true);
+  int st = check_shape(B, H, N, D, true, true);
   if (st != FA_OK) return st;
   if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return FA_ERR_ALIGN;
   fa::BwdLaunch a{};
@@ -236,7 +236,7 @@ static int bwd_common(const void* q, const void* k, const void* v, const void* d
                       size_t workspace_bytes, int B, int H, int N, int D, float scale, int causal, int q_box_rows,
                       bool f16, fa::BwdLaunch* a) {
   if (!q || !k || !v || !dO) return FA_ERR_NULL;
-  int st = check_shape(B, H, N, D, true);
+  int st = check_shape(B, H, N, D, true, true);
   if (st != FA_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO)) return FA_ERR_ALIGN;
   if ((st = workspace_views(const_cast<void*>(workspace), workspace_bytes, B, H, N, D, a)) != FA_OK) return st;
@@ -288,7 +288,7 @@ static int bwd16(const void* q, const void* k, const void* v, const void* o, con
                  void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int D,
                  float scale, int causal, void* stream, bool f16) {
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_NULL;
-  int st = check_shape(B, H, N, D, true);
+  int st = check_shape(B, H, N, D, true, true);
   if (st != FA_OK) return st;
   if (!workspace || workspace_bytes < fa_bwd_workspace_size(B, H, N, D)) return FA_ERR_WORKSPACE;
   // Validate everything the three stages will check, so that an error launches nothing.

@@ -29,21 +29,12 @@
 #include <math_constants.h>
 #include <type_traits>
 
+#include "bwd_common.cuh"
 #include "fa_internal.h"
 #include "sm100_ptx.cuh"
 
 namespace fa {
 namespace {
-
-// 640 threads: warp 0 loads, warp 1 issues MMAs, warps 4-19 are four warpgroups that
-// share the element-wise work (no row reduction is needed in the backward, so the
-// columns of a tile can be split across warpgroups to hide more latency).
-constexpr int kThreads = 640;
-constexpr float kLog2e = 1.44269504088896340736f;
-// Of every 8 pairs of exponentials, this many go to the FMA-pipe polynomial
-// (exp2_poly2) and the rest to the MUFU unit, which alone would bound the softmax.
-constexpr int kPolyPer8 = 2;
-__device__ __forceinline__ bool poly_pair(int c2) { return (c2 & 7) >= 8 - kPolyPer8; }
 
 // ----------------------------------------------------------------------------- stage 1
 // kLanesPerRow lanes per row (a power of two, 8 * kLanesPerRow >= D), each reading 8
@@ -78,65 +69,6 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint16_t* __r
     ws_delta[prow] = acc;
     ws_nl[prow] = real ? -lse[row] * kLog2e : -CUDART_INF_F;
   }
-}
-
-// ----------------------------------------------------------------------------- shared helpers
-// A tile of `rows` rows x D 16-bit values in shared memory, stored as D/64 boxes of rows x 128 bytes
-// in the TMA 128-byte-swizzled layout.
-template <int D, int ROWS>
-struct Tile {
-  static constexpr int kBox = ROWS * 128;
-  static constexpr int kNBox = D / 64;
-  static constexpr int kBytes = kBox * kNBox;
-};
-
-// Copies 64 columns (box `box`) of this thread's fp32 accumulator row in tensor memory,
-// times `mul`, as bf16 (fp16 when F16) into row r of that box of a 128-row staging tile in the TMA
-// 128-byte-swizzled layout.
-template <int D, bool F16>
-__device__ __forceinline__ void stage_box_16(uint32_t tacc, int box, float mul, uint8_t* stage, int r) {
-#pragma unroll
-  for (int cc = 2 * box; cc < 2 * box + 2; ++cc) {
-    uint32_t o[32];
-    tmem_ld32(tacc + cc * 32, o);
-    tmem_ld_wait();
-    reg_fence(o);
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const int chunk = (cc & 1) * 4 + q4;
-      uint4 v;
-      v.x = pack16<F16>(__uint_as_float(o[8 * q4 + 0]) * mul, __uint_as_float(o[8 * q4 + 1]) * mul);
-      v.y = pack16<F16>(__uint_as_float(o[8 * q4 + 2]) * mul, __uint_as_float(o[8 * q4 + 3]) * mul);
-      v.z = pack16<F16>(__uint_as_float(o[8 * q4 + 4]) * mul, __uint_as_float(o[8 * q4 + 5]) * mul);
-      v.w = pack16<F16>(__uint_as_float(o[8 * q4 + 6]) * mul, __uint_as_float(o[8 * q4 + 7]) * mul);
-      *reinterpret_cast<uint4*>(stage + box * Tile<D, 128>::kBox + r * 128 + ((chunk ^ (r & 7)) << 4)) = v;
-    }
-  }
-}
-
-// One warp stores its 32 staged rows of box `box` with the TMA (tensor map box:
-// 64 x 32 x 1); rows at or past n_rows are skipped (or clipped by the hardware).
-template <int D>
-__device__ __forceinline__ void store_warp_box(const CUtensorMap* tm, uint32_t stage_s, int box, int wrow, int row0,
-                                               int bh, int lane, int n_rows) {
-  fence_async_smem();
-  __syncwarp();
-  if (lane == 0 && row0 + wrow < n_rows) {
-    tma_store_3d(tm, stage_s + box * Tile<D, 128>::kBox + wrow * 128, box * 64, row0 + wrow, bh);
-    bulk_commit();
-    bulk_wait_read0();
-  }
-  __syncwarp();
-}
-
-// K-major operand slice for K-step kk (16 values = 32 bytes) of a swizzled tile with box size `box`.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile, int kk, int box) {
-  return sdesc_sw128(tile + (kk >> 2) * box + (kk & 3) * 32, 16, 1024);
-}
-// MN-major operand slice for K-step kk (16 rows of 128 bytes) of a swizzled tile whose
-// 64-column boxes are `box` bytes apart.
-__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t tile, int kk, int box) {
-  return sdesc_sw128(tile + kk * 2048, box, 1024);
 }
 
 // ----------------------------------------------------------------------------- stage 2: dK, dV
@@ -175,12 +107,6 @@ struct DkdvSmem {
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
-// Tensor-memory column of the packed 16-bit pairs for K-step kk (16 queries) of the
-// P^T (base 0) or dS^T (base 128) operand: queries [32g, 32g+32) are packed into
-// columns base + [32g, 32g+16).
-__device__ __forceinline__ uint32_t packed_col(uint32_t base, int kk) {
-  return base + 32 * (kk >> 1) + 8 * (kk & 1);
-}
 
 template <int D, bool CAUSAL, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -791,7 +717,8 @@ cudaError_t dq_impl(const BwdLaunch& a, cudaStream_t stream) {
 template <bool F16>
 cudaError_t preprocess_typed(const BwdLaunch& a, cudaStream_t stream) {
   if (a.D <= 32) return preprocess_impl<4, F16>(a, stream);
-  return a.D <= 64 ? preprocess_impl<8, F16>(a, stream) : preprocess_impl<16, F16>(a, stream);
+  if (a.D <= 64) return preprocess_impl<8, F16>(a, stream);
+  return a.D <= 128 ? preprocess_impl<16, F16>(a, stream) : preprocess_impl<32, F16>(a, stream);
 }
 
 template <bool F16>
@@ -815,10 +742,12 @@ cudaError_t launch_bwd_preprocess(const BwdLaunch& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_bwd_dkdv(const BwdLaunch& a, cudaStream_t stream) {
+  if (a.D == 256) return launch_bwd_dkdv_d256(a, stream);
   return a.f16 ? dkdv_typed<true>(a, stream) : dkdv_typed<false>(a, stream);
 }
 
 cudaError_t launch_bwd_dq(const BwdLaunch& a, cudaStream_t stream) {
+  if (a.D == 256) return launch_bwd_dq_d256(a, stream);
   return a.f16 ? dq_typed<true>(a, stream) : dq_typed<false>(a, stream);
 }
 

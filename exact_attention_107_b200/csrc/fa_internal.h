@@ -49,5 +49,8 @@ struct BwdLaunch {
 cudaError_t launch_bwd_preprocess(const BwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_bwd_dkdv(const BwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_bwd_dq(const BwdLaunch& a, cudaStream_t stream);
+// Head dimension 256 (fa_bwd_d256_sm100.cu): two CTAs per tile, one per half of D.
+cudaError_t launch_bwd_dkdv_d256(const BwdLaunch& a, cudaStream_t stream);
+cudaError_t launch_bwd_dq_d256(const BwdLaunch& a, cudaStream_t stream);
 
 }  // namespace fa

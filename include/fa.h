@@ -27,9 +27,9 @@
  *     host synchronisation.
  *   - Supported: B, H, N >= 1; D in {32, 64, 96, 128} for bf16 and fp16 (32
  *     and 96 run the 64- and 128-column kernels on zero-filled columns, so
- *     they cost what 64 and 128 cost), and D = 256 for the bf16 / fp16 forward
- *     only (the backward returns FA_ERR_HEADDIM for it); D in {32, 64, 128}
- *     for fp32; Nq == Nk == N; causal in {0, 1}; ceil(N/256)*B*H < 2^31 (and
+ *     they cost what 64 and 128 cost), and D = 256 (forward: one query tile
+ *     per CTA; backward: two CTAs per tile, one per half of D); D in
+ *     {32, 64, 128} for fp32; Nq == Nk == N; causal in {0, 1}; ceil(N/256)*B*H < 2^31 (and
  *     B*H <= 65535 for fa_fwd_f32).
  *   - Return value: FA_OK (0) or an fa_status code.  Arguments are validated
  *     before anything is launched; on an error nothing is launched and no

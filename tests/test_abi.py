@@ -42,7 +42,7 @@ def test_workspace_size():
     assert fa.fa_bwd_workspace_size(2, 3, 129, 64) == 2 * 6 * 256 * 4
     assert fa.fa_bwd_workspace_size(1, 1, 128, 96) == 2 * 128 * 4
     assert fa.fa_bwd_workspace_size(1, 1, 128, 80) == 0          # unsupported D
-    assert fa.fa_bwd_workspace_size(1, 1, 128, 256) == 0         # D = 256: forward only
+    assert fa.fa_bwd_workspace_size(1, 1, 128, 256) == 2 * 128 * 4
 
 
 def test_noalloc_capacity_check_needs_no_gpu():
@@ -91,7 +91,7 @@ def test_bwd_rejects_bad_arguments():
     assert lib.fa_bwd(*args[:8], U, P, ws, 1, 2, 256, 64, 0.125, 0, None) == 4
     assert lib.fa_bwd(*args[:3], Z, *args[4:], P, ws, 1, 2, 256, 64, 0.125, 0, None) == 1
     assert lib.fa_bwd(*args, P, ws, 1, 2, 256, 80, 0.125, 0, None) == 3
-    assert lib.fa_bwd(*args, P, ws, 1, 2, 256, 256, 0.125, 0, None) == 3     # D = 256: forward only
+    assert lib.fa_bwd(*args, P, ws, 1, 2, 256, 192, 0.125, 0, None) == 3
     ws1 = lib.fa_bwd_workspace_size(1, 1, 128, 64)
     assert ws1 == 2 * 128 * 4
     assert lib.fa_bwd_dq(P, P, P, P, P, ws1, Z, 1, 1, 128, 64, 0.1, 0, None) == 1

@@ -16,7 +16,7 @@ SHAPES = [
     (1, 2, 128, 64, False), (1, 2, 256, 128, True), (2, 3, 384, 64, True),
     (1, 1, 1, 64, False), (1, 2, 200, 64, True), (1, 2, 129, 128, True),
     (1, 1, 300, 128, False), (1, 4, 1024, 128, True), (1, 3, 1000, 64, False),
-    (1, 2, 384, 96, True), (1, 2, 300, 32, False),
+    (1, 2, 384, 96, True), (1, 2, 300, 32, False), (1, 2, 384, 256, True), (1, 1, 200, 256, False),
 ]
 
 

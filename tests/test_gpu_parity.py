@@ -93,11 +93,18 @@ def test_forward_head_dim_256_growing_max(causal):
     check_fwd(O.cpu(), lse.cpu(), ref_O, ref_lse)
 
 
-def test_backward_head_dim_256_is_rejected():
-    q = torch.zeros(1, 1, 128, 256, dtype=torch.bfloat16, device="cuda")
-    lse = torch.zeros(1, 1, 128, device="cuda")
-    with pytest.raises(fa.FAError):
-        fa.attention_backward(q, q, q, q, lse, q, 0.0625, False)
+D256_BWD = [(1, 2, 256, 256, False), (1, 2, 384, 256, True), (2, 1, 200, 256, True), (1, 1, 1, 256, False),
+            (1, 2, 1000, 256, False), (1, 2, 640, 256, True)]
+
+
+@pytest.mark.parametrize("B,H,N,D,causal", D256_BWD)
+def test_backward_head_dim_256(B, H, N, D, causal):
+    """The two-CTA-per-tile backward (each CTA owns one half of D)."""
+    w, (q, k, v, do) = _small(B, H, N, D, causal)
+    got = gpu_fwd_bwd(q, k, v, do, w.softmax_scale, causal)
+    ref = oracle.attention_backward(q, k, v, do, w.softmax_scale, causal)
+    check_fwd(got["O"], got["lse"], ref["O"], ref["lse"], (B, H, N, D, causal))
+    check_grads(got, ref, (B, H, N, D, causal))
 
 
 @pytest.mark.parametrize("D,causal", [(64, False), (128, True)])
