@@ -278,21 +278,26 @@ def attention_fwd_bwd_from_host(q_h, k_h, v_h, do_h, scale: float, causal: bool,
     device, run forward and backward, and copy O, lse, dQ, dK, dV back to `out`
     (pinned host tensors, allocated when None).  Returns (out, h2d_bytes, d2h_bytes)."""
     B, H, N, D = q_h.shape
+    dtype = q_h.dtype
+    if dtype not in (torch.bfloat16, torch.float16):
+        raise TypeError(f"q must be bfloat16 or float16, got {dtype}")
     if dev_bufs is None:
         dev = torch.device("cuda")
-        dev_bufs = {n: torch.empty(B, H, N, D, device=dev, dtype=torch.bfloat16)
+        dev_bufs = {n: torch.empty(B, H, N, D, device=dev, dtype=dtype)
                     for n in ("q", "k", "v", "do", "o", "dq", "dk", "dv")}
         dev_bufs["lse"] = torch.empty(B, H, N, device=dev, dtype=torch.float32)
         dev_bufs["ws"] = torch.empty(fa_bwd_workspace_size(B, H, N, D), device=dev, dtype=torch.uint8)
     if out is None:
-        out = {n: torch.empty(B, H, N, D, dtype=torch.bfloat16).pin_memory() for n in ("o", "dq", "dk", "dv")}
+        out = {n: torch.empty(B, H, N, D, dtype=dtype).pin_memory() for n in ("o", "dq", "dk", "dv")}
         out["lse"] = torch.empty(B, H, N, dtype=torch.float32).pin_memory()
     d = dev_bufs
     for n, h in (("q", q_h), ("k", k_h), ("v", v_h), ("do", do_h)):
+        if h.dtype != dtype or d[n].dtype != dtype:
+            raise TypeError(f"{n}: every input and device buffer must be {dtype}")
         d[n].copy_(h, non_blocking=True)
-    fa_fwd(d["q"], d["k"], d["v"], d["o"], d["lse"], scale, causal, stream)
-    fa_bwd(d["q"], d["k"], d["v"], d["o"], d["do"], d["lse"], d["dq"], d["dk"], d["dv"], d["ws"], scale, causal,
-           stream)
+    fwd, bwd = (fa_fwd_f16, fa_bwd_f16) if dtype == torch.float16 else (fa_fwd, fa_bwd)
+    fwd(d["q"], d["k"], d["v"], d["o"], d["lse"], scale, causal, stream)
+    bwd(d["q"], d["k"], d["v"], d["o"], d["do"], d["lse"], d["dq"], d["dk"], d["dv"], d["ws"], scale, causal, stream)
     for n in ("o", "lse", "dq", "dk", "dv"):
         out[n].copy_(d[n], non_blocking=True)
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, do_h))

@@ -43,3 +43,21 @@ def test_pipelined_steps_match_direct_calls(dtype):
     got = {"O": outs[0]["o"], "lse": outs[0]["lse"], "dQ": outs[0]["dq"], "dK": outs[0]["dk"], "dV": outs[0]["dv"]}
     check_fwd(got["O"], got["lse"], ref["O"], ref["lse"])
     check_grads(got, ref)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_single_step_from_host_matches_direct_calls(dtype):
+    B, H, N, D, causal = 1, 2, 384, 64, False
+    q, k, v, do = workloads.make_inputs(workloads.custom("host", B, H, N, D, causal, dtype=dtype, seed=7),
+                                        with_grad_out=True)
+    scale = D ** -0.5
+    out, h2d, d2h = fa.attention_fwd_bwd_from_host(*(t.pin_memory() for t in (q, k, v, do)), scale, causal)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status(reset=True) == 0
+    assert out["o"].dtype == q.dtype and h2d == 4 * q.numel() * q.element_size()
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = fa.attention_forward(qd, kd, vd, scale, causal)
+    dq, dk, dv = fa.attention_backward(qd, kd, vd, o, lse, dod, scale, causal)
+    torch.cuda.synchronize()
+    for name, ref in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+        assert torch.equal(out[name], ref.cpu()), name
