@@ -17,7 +17,7 @@ namespace {
 constexpr int kThreads = 640;
 constexpr float kLog2e = 1.44269504088896340736f;
 // Of every 8 pairs of exponentials, this many go to the FMA-pipe polynomial
-// (exp2_poly2) and the rest to the MUFU unit, which alone would bound the softmax.
+// (exp2_poly2) and the rest to the MUFU unit (1/8 to 3/8 measure within 1% of each other).
 constexpr int kPolyPer8 = 2;
 __device__ __forceinline__ bool poly_pair(int c2) { return (c2 & 7) >= 8 - kPolyPer8; }
 
