@@ -1,24 +1,27 @@
-"""Benchmark: attention TFLOPS, forward + backward, bf16, on B200.
+"""Benchmark: attention TFLOPS, forward and forward + backward, on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-One step = the whole hot path on one batch: fa_fwd (forward, saves lse), then
-the backward's three stages (delta preprocess, dK/dV kernel, dQ kernel), all
-through the C ABI.  Default workload: long-context causal attention,
-B1 H8 N65536 D128 (the spec D=128, N>=4096 configuration).
+One step = the whole hot path on one batch, through the C ABI: the forward (fa_fwd,
+or fa_fwd_f32 for the fp32 workload) and, for workloads with a backward, its three
+kernels (row statistics + accumulator zeroing, the fused dK/dV/dQ kernel, dQ finish).
+Default workload: long-context causal attention, B1 H8 N65536 D128 (the D=128,
+N>=4096 configuration the metric is quoted on); the other four workloads (fp32
+forward, bf16 forward, non-causal and GPT-2-style fwd+bwd) run with --workload.
 
 Throughput accounting (algorithmic, attention convention):
     F_fwd = 4 * B * H * N^2 * D, halved when causal
-    value = 2.5 * F_fwd / (t_fwd + t_bwd)            ("metric-as-stated", the headline)
-    detail.fwd_tflops = F_fwd / t_fwd, detail.bwd_tflops = 2.5 * F_fwd / t_bwd,
-    detail.fwd_bwd_tflops_3_5x = 3.5 * F_fwd / (t_fwd + t_bwd)
-Inputs (Q, K, V, dO: 4 x 128 MiB for the default workload) are larger than the
-126 MB L2, so no flush is needed between steps.  With N GPUs (torchrun), every
-rank runs its own copy of the workload (independent batch/head shards, no
+    value = 2.5 * F_fwd / (t_fwd + t_bwd)   for workloads with a backward (the headline)
+          = F_fwd / t_fwd                   for forward-only workloads
+    detail: fwd_tflops, bwd_tflops = 2.5 F_fwd / t_bwd, fwd_bwd_tflops_3_5x = 3.5 F_fwd / (t_fwd + t_bwd)
+Cold L2: when a workload's inputs are smaller than twice the 126 MB L2, a 256 MiB
+buffer is written between steps (outside the timed spans); larger inputs evict L2
+by themselves.  The `l2` field of `config` says which.  With N GPUs (torchrun),
+every rank runs its own copy of the workload (independent batch/head shards, no
 collective on the data path): weak scaling, time = max over ranks.
 
---impl reference times the fp64 CPU oracle (the only reference this method has:
-the pages ship no code) on a bounded sample of the same workload.
+--impl reference times the fp64 CPU oracle (the only reference this method has: the
+pages ship no code) on a bounded sample of the same workload.
 """
 from __future__ import annotations
 
@@ -26,7 +29,6 @@ import argparse
 import hashlib
 import json
 import os
-import re
 import statistics
 import subprocess
 import sys
@@ -40,29 +42,38 @@ sys.path.insert(0, str(ROOT))
 
 import workloads  # noqa: E402
 
+METRIC = "attention TFLOPS fwd and fwd+bwd (bf16, 1 B200); % of dense BF16 tensor peak"
 PEAKS_FILE = ROOT / "MEASURED_PEAKS.json"
-TRAFFIC_FILE = ROOT / "profiles" / "dram_traffic.md"
+TRAFFIC_FILE = ROOT / "profiles" / "dram_traffic.json"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# NVIDIA's published dense BF16 tensor throughput of one B200 (the datasheet's 4.5 PFLOP/s
+# is with 2:4 sparsity), reported as a third denominator.
+DATASHEET_BF16_TFLOPS = 2250.0
+# Plain fp32 FFMA peak, for the fp32 path: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz.
+FP32_FFMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+L2_BYTES = 126e6
+FLUSH_BYTES = 256 << 20
 KERNEL_SOURCES = {
     "fwd": "exact_attention_107_b200/csrc/fa_fwd_sm100.cu",
-    "bwd_dkdv": "exact_attention_107_b200/csrc/fa_bwd_sm100.cu",
-    "bwd_dq": "exact_attention_107_b200/csrc/fa_bwd_sm100.cu",
+    "fwd_f32": "exact_attention_107_b200/csrc/fa_fwd_f32.cu",
+    "bwd_main": "exact_attention_107_b200/csrc/fa_bwd_fused_sm100.cu",
+    "bwd_finish": "exact_attention_107_b200/csrc/fa_bwd_fused_sm100.cu",
     "bwd_pre": "exact_attention_107_b200/csrc/fa_bwd_sm100.cu",
 }
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="c5_long_causal")
+    ap.add_argument("--workload", default="c5_long_causal", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shape", default=None,
-                    help="B,H,N,D,causal: a custom workload of the same recipe (profiling small cases)")
-    a = ap.parse_args()
+                    help="B,H,N,D,causal: a custom bf16 fwd+bwd workload of the same recipe (profiling small cases)")
+    a = ap.parse_args(argv)
     if a.shape:
         B, H, N, D, c = (int(x) for x in a.shape.split(","))
         name = f"custom_B{B}_H{H}_N{N}_D{D}_{'causal' if c else 'full'}"
@@ -73,8 +84,7 @@ def parse_args():
 
 def load_peaks():
     if PEAKS_FILE.exists():
-        d = json.loads(PEAKS_FILE.read_text())
-        return d, "measured"
+        return json.loads(PEAKS_FILE.read_text()), "measured"
     return dict(FALLBACK_PEAKS), "fallback"
 
 
@@ -83,15 +93,52 @@ def source_sha(rel: str) -> str:
 
 
 def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch recorded from an ncu capture, if the kernel source is unchanged since."""
+    """DRAM bytes per launch recorded from an ncu capture (profiles/dram_traffic.json), if the
+    kernel source is unchanged since the capture; None otherwise."""
     if not TRAFFIC_FILE.exists():
         return None
-    for line in TRAFFIC_FILE.read_text().splitlines():
-        m = re.match(r"\|\s*(\w+)\s*\|\s*(\w+)\s*\|\s*([0-9.eE+]+)\s*\|\s*([0-9a-f]{12})\s*\|", line)
-        if m and m.group(1) == kernel and m.group(2) == workload:
-            if m.group(4) == source_sha(KERNEL_SOURCES[kernel]):
-                return float(m.group(3))
+    for e in json.loads(TRAFFIC_FILE.read_text()).get("entries", []):
+        if e.get("kernel") == kernel and e.get("workload") == workload:
+            if e.get("source_sha") == source_sha(KERNEL_SOURCES[kernel]):
+                return float(e["bytes_per_launch"])
     return None
+
+
+def input_bytes(w) -> int:
+    elem = 4 if w.dtype == "fp32" else 2
+    return (4 if w.backward else 3) * w.B * w.H * w.N * w.D * elem
+
+
+def needs_flush(w) -> bool:
+    """Inputs smaller than twice the L2 could stay cached between steps: flush."""
+    return input_bytes(w) < 2 * L2_BYTES
+
+
+def l2_label(w) -> str:
+    mib = input_bytes(w) / 2**20
+    if needs_flush(w):
+        return f"inputs {mib:.0f} MiB < 2 x L2: a {FLUSH_BYTES >> 20} MiB buffer is written before every step (untimed)"
+    return f"inputs {mib:.0f} MiB > 2 x L2 (126 MB): no flush needed"
+
+
+def kernel_names(w):
+    if not w.backward:
+        return ("fwd_f32",) if w.dtype == "fp32" else ("fwd",)
+    return ("fwd", "bwd_pre", "bwd_main", "bwd_finish")
+
+
+def algorithmic_flops(w):
+    """Algorithmic FLOPs per launch of each kernel: the forward's two GEMMs (F_fwd) and the
+    backward's five (QK^T, dO V^T, P^T dO, dS^T Q, dS K: 2.5 F_fwd, all in the fused kernel)."""
+    f = w.fwd_flops()
+    return {"fwd": f, "fwd_f32": f, "bwd_pre": 0.0, "bwd_main": 2.5 * f, "bwd_finish": 0.0}
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 # ----------------------------------------------------------------------------- multi-rank helpers
@@ -112,6 +159,11 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
 def whole_job_tflops(world: int, flops_per_rank: float, ms: float) -> float:
     """Aggregate throughput: the work of all ranks over the slowest rank's time."""
     return world * flops_per_rank / (ms * 1e-3) / 1e12
+
+
+def step_flops(w) -> float:
+    """FLOPs of one step by the metric's count."""
+    return (2.5 if w.backward else 1.0) * w.fwd_flops()
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -177,34 +229,40 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     # each rank holds its own shard of heads: same shapes, its own seed
     wr = workloads.custom(w.name, w.B, w.H, w.N, w.D, w.causal, dtype=w.dtype, seed=shard_seed(w.seed, rank),
-                          qkv_std=w.qkv_std, scale=w.scale, backward=True)
-    q_h, k_h, v_h, do_h = workloads.make_inputs(wr, with_grad_out=True)
+                          qkv_std=w.qkv_std, scale=w.scale, backward=w.backward)
+    q_h, k_h, v_h, do_h = workloads.make_inputs(wr, with_grad_out=w.backward)
     B, H, N, D = q_h.shape
     scale, causal = w.softmax_scale, w.causal
-    q, k, v, do = (t.to(dev) for t in (q_h, k_h, v_h, do_h))
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
     o = torch.empty_like(q)
     lse = torch.empty(B, H, N, device=dev, dtype=torch.float32)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, D), device=dev, dtype=torch.uint8)
+    if w.backward:
+        do = do_h.to(dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, D), device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream(dev)
-
-    names = ("fwd", "bwd_pre", "bwd_dkdv", "bwd_dq")
+    flush = torch.empty(FLUSH_BYTES, device=dev, dtype=torch.uint8) if needs_flush(w) else None
+    names = kernel_names(w)
+    fwd = fa.fa_fwd_f32 if w.dtype == "fp32" else fa.fa_fwd
 
     def step(ev=None):
+        if flush is not None:
+            flush.fill_(1)                 # evict L2 (not timed: the spans start after it)
         if ev is not None:
             ev[0].record(stream)
-        fa.fa_fwd(q, k, v, o, lse, scale, causal, stream)
+        fwd(q, k, v, o, lse, scale, causal, stream)
         if ev is not None:
             ev[1].record(stream)
-        fa.fa_bwd_preprocess(o, do, lse, ws, stream)
-        if ev is not None:
-            ev[2].record(stream)
-        fa.fa_bwd_dkdv(q, k, v, do, ws, dk, dv, scale, causal, stream)
-        if ev is not None:
-            ev[3].record(stream)
-        fa.fa_bwd_dq(q, k, v, do, ws, dq, scale, causal, stream)
-        if ev is not None:
-            ev[4].record(stream)
+        if w.backward:
+            fa.fa_bwd_preprocess(o, do, lse, ws, stream)
+            if ev is not None:
+                ev[2].record(stream)
+            fa.fa_bwd_dkdvdq(q, k, v, do, ws, dk, dv, scale, causal, stream)
+            if ev is not None:
+                ev[3].record(stream)
+            fa.fa_bwd_dq_finish(ws, dq, scale, stream)
+            if ev is not None:
+                ev[4].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -212,36 +270,31 @@ def run_ours(args, rank, world, local_rank):
     if fa.fa_device_status(reset=True) != 0:
         raise RuntimeError("device status error during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local_rank) as clk:
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(stream)
         for i in range(args.steps):
             step(evs[i])
-        t_end.record(stream)
         torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
     per = {n: [evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(args.steps)] for j, n in enumerate(names)}
+    spans = [evs[i][0].elapsed_time(evs[i][-1]) for i in range(args.steps)]
     status = fa.fa_device_status(reset=True)
     if status != 0:
         raise RuntimeError(f"device status {status} after timed region")
-
-    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
+    elapsed_ms = max_over_ranks(sum(spans), world, dev)
 
     # ---------------------------------------------------------------- end-to-end from host buffers
     e2e = None
     if not args.no_e2e:
-        # Every step uploads its inputs from pinned host memory and downloads O, lse, dQ,
-        # dK, dV; HostStepPipeline overlaps step i's kernels with the copies of its
-        # neighbours (two device buffer sets, separate copy streams).
-        pinned = [t.pin_memory() for t in (q_h, k_h, v_h, do_h)]
-        pipe = fa.HostStepPipeline(B, H, N, D, dtype=q.dtype, device=dev)
+        # Every step uploads its inputs from pinned host memory and downloads its results
+        # (O, lse and, with a backward, dQ, dK, dV); HostStepPipeline overlaps step i's
+        # kernels with the copies of its neighbours (two device buffer sets, copy streams).
+        pinned = [t.pin_memory() for t in (q_h, k_h, v_h)] + [do_h.pin_memory() if w.backward else None]
+        pipe = fa.HostStepPipeline(B, H, N, D, dtype=q.dtype, device=dev, backward=w.backward)
         outs = [pipe.host_outputs() for _ in range(pipe.depth)]
         for i in range(max(1, args.warmup)):
             pipe.submit(*pinned, outs[i % pipe.depth], scale, causal)
@@ -261,26 +314,49 @@ def run_ours(args, rank, world, local_rank):
     return w, per, elapsed_ms, clk.summary(), e2e
 
 
-def cpu_baseline(w, rows: int = 8192, heads=None, repeats: int = 1):
-    """The fp64 oracle, as it stands, on a bounded sample of the workload: the causal
-    (or leading, if non-causal) rows x rows block of each sampled head, forward and
-    backward.  Returns (TFLOPS by the metric's count, seconds, description)."""
+def cpu_baseline(w, full: bool, rows: int = 8192, heads=None, repeats: int = 1):
+    """The fp64 oracle, as it stands, on the host cores: the whole workload (full), or a
+    bounded sample of it, the causal (or leading) rows x rows block of each sampled head.
+    Forward and backward where the workload has a backward.  Returns (TFLOPS by the
+    metric's count, seconds, description)."""
     import oracle
 
-    q, k, v, do = workloads.make_inputs(w, with_grad_out=True)
-    n = min(rows, w.N)
+    q, k, v, do = workloads.make_inputs(w, with_grad_out=w.backward)
+    n = w.N if full else min(rows, w.N)
     heads = list(range(w.B * w.H)) if heads is None else heads
+    mult = 2.5 if w.backward else 1.0
     t0 = time.time()
     flops = 0.0
     for _ in range(repeats):
+        if full and heads == list(range(w.B * w.H)):
+            if w.backward:
+                oracle.attention_backward(q, k, v, do, w.softmax_scale, w.causal)
+            else:
+                oracle.attention_forward(q, k, v, w.softmax_scale, w.causal)
+            flops += mult * w.fwd_flops()
+            continue
         for bh in heads:
             b, h = divmod(bh, w.H)
             sl = (slice(b, b + 1), slice(h, h + 1), slice(0, n))
-            oracle.attention_backward(q[sl], k[sl], v[sl], do[sl], w.softmax_scale, w.causal)
-            flops += 2.5 * 4.0 * n * n * w.D / (2.0 if w.causal else 1.0)
+            if w.backward:
+                oracle.attention_backward(q[sl], k[sl], v[sl], do[sl], w.softmax_scale, w.causal)
+            else:
+                oracle.attention_forward(q[sl], k[sl], v[sl], w.softmax_scale, w.causal)
+            flops += mult * 4.0 * n * n * w.D / (2.0 if w.causal else 1.0)
     dt = time.time() - t0
-    desc = f"fp64 oracle fwd+bwd on the first {n} of {w.N} rows of {len(heads)} head(s), x{repeats}"
+    what = "fwd+bwd" if w.backward else "fwd"
+    if full:
+        desc = f"fp64 oracle {what} on the whole workload"
+    else:
+        desc = f"fp64 oracle {what} on the first {n} of {w.N} rows of {len(heads)} head(s)"
+    desc += f", x{repeats}; BLAS threads {torch.get_num_threads()}"
     return flops / dt / 1e12, dt, desc
+
+
+def oracle_runs_full(w) -> bool:
+    """The oracle is timed on the whole workload where that takes seconds (every workload but
+    the long-context one, whose S matrix per head alone is 32 GiB in fp64)."""
+    return w.N <= 8192
 
 
 def main():
@@ -289,27 +365,30 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = workloads.WORKLOADS[args.workload]
-    metric = "attention TFLOPS fwd+bwd (bf16, 1 B200)"
+    dtype = "f32" if w.dtype == "fp32" else w.dtype
 
     if args.impl == "reference":
         if rank != 0:
             return
+        full = oracle_runs_full(w)
+        heads = None if full else [0]
         tflops_s = []
         for _ in range(args.warmup):
-            cpu_baseline(w, heads=[0])
+            cpu_baseline(w, full, heads=heads)
         t_all = 0.0
+        desc = ""
         for _ in range(args.steps):
-            v, dt, desc = cpu_baseline(w, heads=[0])
+            v, dt, desc = cpu_baseline(w, full, heads=heads)
             tflops_s.append(v)
             t_all += dt
         value = statistics.median(tflops_s)
-        cores = torch.get_num_threads()
         print(json.dumps({
-            "impl": "reference", "metric": metric, "value": value, "unit": "TFLOPS", "n_gpus": 1,
+            "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * t_all / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {**w.describe(), "sample": desc},
-            "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": desc},
+            "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cpu_cores(), "kind": "oracle",
+                             "sample": desc},
             "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }))
         return
@@ -326,50 +405,59 @@ def main():
 
     f_fwd = w.fwd_flops()
     ms_step = elapsed_ms / args.steps
-    value = whole_job_tflops(world, 2.5 * f_fwd, ms_step)
+    value = whole_job_tflops(world, step_flops(w), ms_step)
     mean = {n: statistics.mean(v) for n, v in per.items()}
     peaks, peak_kind = load_peaks()
     peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     peak_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    # Algorithmic FLOPs per launch of each kernel (the backward's five GEMMs: the dK/dV
-    # kernel does S, dP, dV, dK = 2 * F_fwd; the dQ kernel's algorithmic share is the
-    # dQ GEMM = 0.5 * F_fwd, its recomputed S and dP are extra work).
-    alg = {"fwd": f_fwd, "bwd_dkdv": 2.0 * f_fwd, "bwd_dq": 0.5 * f_fwd, "bwd_pre": 0.0}
-    dom = max(("fwd", "bwd_dkdv", "bwd_dq"), key=lambda n: mean[n])
+    alg = algorithmic_flops(w)
+    timed = [n for n in per if alg[n] > 0]
+    dom = max(timed, key=lambda n: mean[n])
     achieved = alg[dom] / (mean[dom] * 1e-3) / 1e12
-    detail = {
-        "t_fwd_ms": mean["fwd"], "t_bwd_ms": mean["bwd_pre"] + mean["bwd_dkdv"] + mean["bwd_dq"],
-        "t_kernels_ms": mean,
-        "fwd_tflops": f_fwd / (mean["fwd"] * 1e-3) / 1e12,
-        "bwd_tflops": 2.5 * f_fwd / ((mean["bwd_pre"] + mean["bwd_dkdv"] + mean["bwd_dq"]) * 1e-3) / 1e12,
-        "fwd_bwd_tflops_3_5x": whole_job_tflops(world, 3.5 * f_fwd, ms_step),
-    }
-    detail["fwd_frac_of_burst_peak"] = detail["fwd_tflops"] / peak_burst
-    detail["fwd_bwd_frac_of_burst_peak"] = value / world / peak_burst
+    t_fwd = mean[kernel_names(w)[0]]
+    t_bwd = sum(mean[n] for n in ("bwd_pre", "bwd_main", "bwd_finish") if n in mean)
+    detail = {"t_fwd_ms": t_fwd, "t_kernels_ms": mean, "fwd_tflops": f_fwd / (t_fwd * 1e-3) / 1e12}
+    if w.backward:
+        detail.update({"t_bwd_ms": t_bwd, "bwd_tflops": 2.5 * f_fwd / (t_bwd * 1e-3) / 1e12,
+                       "fwd_bwd_tflops_3_5x": whole_job_tflops(world, 3.5 * f_fwd, ms_step)})
+    if w.dtype != "fp32":
+        detail["fwd_frac_of_burst_peak"] = detail["fwd_tflops"] / peak_burst
+        detail["value_frac_of_burst_peak"] = value / world / peak_burst
+        detail["value_frac_of_datasheet_peak"] = value / world / DATASHEET_BF16_TFLOPS
+    if w.dtype == "fp32":
+        roofline = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": FP32_FFMA_TFLOPS,
+                    "unit": "TFLOP/s", "frac": achieved / FP32_FFMA_TFLOPS,
+                    "peak_kind": "derived fp32 FFMA peak: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz",
+                    "traffic": recorded_traffic(dom, w.name)}
+    else:
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s",
+                    "frac": achieved / peak_burst,
+                    "peak_kind": f"{peak_kind} bf16 burst (kernel timed on its own launches)",
+                    "frac_of_sustained": achieved / peak_sust,
+                    "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS,
+                    "traffic": recorded_traffic(dom, w.name)}
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        v, dt, desc = cpu_baseline(w, repeats=3)
-        cpu = {"value": v, "unit": "TFLOPS", "cores": torch.get_num_threads(), "kind": "oracle", "sample": desc,
-               "seconds": dt}
+        full = oracle_runs_full(w)
+        v, dt, desc = cpu_baseline(w, full, repeats=1 if full else 3)
+        cpu = {"value": v, "unit": "TFLOPS", "cores": cpu_cores(), "blas_threads": torch.get_num_threads(),
+               "kind": "oracle", "sample": desc, "seconds": dt}
     out = {
-        "metric": metric, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+        "value_kind": "fwd+bwd (2.5 x F_fwd per step)" if w.backward else "fwd (F_fwd per step)",
         "config": {**w.describe(), "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": "inputs (4 x %d MiB) larger than L2, no flush" % (w.B * w.H * w.N * w.D * 2 >> 20),
-                   "flops": "F_fwd=4BHN^2D/(2 if causal); value=2.5*F_fwd/(t_fwd+t_bwd)"},
-        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak_sust, "unit": "TFLOP/s",
-                     "frac": achieved / peak_sust,
-                     "peak_kind": f"{peak_kind} bf16 sustained (kernel timed inside a long step loop)",
-                     "frac_of_burst": achieved / peak_burst,
-                     "traffic": recorded_traffic(dom, w.name)},
+                   "l2": l2_label(w),
+                   "flops": "F_fwd=4BHN^2D/(2 if causal); value=2.5*F_fwd/(t_fwd+t_bwd) (fwd only: F_fwd/t_fwd)"},
+        "roofline": roofline,
         "cpu_baseline": cpu,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": len(per) * args.steps,
         "clocks": clocks,
         "detail": detail,
     }
     if e2e is not None:
-        out["e2e"] = {"value": whole_job_tflops(world, 2.5 * f_fwd, e2e["ms_per_step"]), "unit": "TFLOPS",
+        out["e2e"] = {"value": whole_job_tflops(world, step_flops(w), e2e["ms_per_step"]), "unit": "TFLOPS",
                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                       "ms_per_step": e2e["ms_per_step"]}
     print(json.dumps(out))

@@ -17,8 +17,12 @@ from ._binding import (  # noqa: F401
     default_scale,
     fa_bwd,
     fa_bwd_f16,
+    fa_bwd_deterministic,
+    fa_bwd_deterministic_workspace_size,
     fa_bwd_dkdv,
+    fa_bwd_dkdvdq,
     fa_bwd_dq,
+    fa_bwd_dq_finish,
     fa_bwd_noalloc,
     fa_bwd_preprocess,
     fa_bwd_workspace_size,
@@ -33,4 +37,4 @@ from ._binding import (  # noqa: F401
     workspace_views,
 )
 
-__version__ = "1.0.0"
+__version__ = "2.0.0"

@@ -20,7 +20,8 @@ LIB_PATH = pathlib.Path(__file__).resolve().with_name("libfa.so")
 SYMBOLS = (
     "fa_fwd", "fa_fwd_f32", "fa_bwd_workspace_size", "fa_bwd", "fa_bwd_preprocess",
     "fa_bwd_dkdv", "fa_bwd_dq", "fa_status_string", "fa_device_status", "fa_version",
-    "fa_bwd_noalloc", "fa_fwd_f16", "fa_bwd_f16",
+    "fa_bwd_noalloc", "fa_fwd_f16", "fa_bwd_f16", "fa_bwd_deterministic",
+    "fa_bwd_deterministic_workspace_size", "fa_bwd_dkdvdq", "fa_bwd_dq_finish",
 )
 
 _lib = None
@@ -46,6 +47,11 @@ def load_library() -> ctypes.CDLL:
     lib.fa_fwd_f16.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
     lib.fa_bwd_workspace_size.restype = sz
+    lib.fa_bwd_deterministic_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_bwd_deterministic_workspace_size.restype = sz
+    lib.fa_bwd_deterministic.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
+    lib.fa_bwd_dkdvdq.argtypes = [vp, vp, vp, vp, vp, sz, vp, vp, i, i, i, i, f, i, vp]
+    lib.fa_bwd_dq_finish.argtypes = [vp, sz, vp, i, i, i, i, f, vp]
     lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
     lib.fa_bwd_f16.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i, i, i, i, f, i, vp]
     lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, vp, sz, i, i, i, i, vp]
@@ -58,7 +64,8 @@ def load_library() -> ctypes.CDLL:
     lib.fa_device_status.argtypes = [i]
     lib.fa_version.argtypes = []
     for name in ("fa_fwd", "fa_fwd_f32", "fa_fwd_f16", "fa_bwd", "fa_bwd_f16", "fa_bwd_preprocess", "fa_bwd_dkdv",
-                 "fa_bwd_dq", "fa_device_status", "fa_version"):
+                 "fa_bwd_dq", "fa_device_status", "fa_version", "fa_bwd_deterministic", "fa_bwd_dkdvdq",
+                 "fa_bwd_dq_finish"):
         getattr(lib, name).restype = i
     _lib = lib
     return lib
@@ -134,10 +141,22 @@ def fa_bwd_workspace_size(B: int, H: int, N: int, D: int) -> int:
     return int(load_library().fa_bwd_workspace_size(B, H, N, D))
 
 
+def fa_bwd_deterministic_workspace_size(B: int, H: int, N: int, D: int) -> int:
+    return int(load_library().fa_bwd_deterministic_workspace_size(B, H, N, D))
+
+
 def fa_bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, causal: bool, stream=None) -> None:
     """dq, dk, dv <- gradients of attention (bf16); workspace: uint8 CUDA tensor of
-    fa_bwd_workspace_size bytes."""
+    fa_bwd_workspace_size bytes.  dQ is summed in fp32 in a run-dependent order."""
     _bwd16("fa_bwd", torch.bfloat16, q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal, stream)
+
+
+def fa_bwd_deterministic(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, causal: bool,
+                         stream=None) -> None:
+    """Bit-reproducible bf16 backward (three stages, no atomics); workspace of at least
+    fa_bwd_deterministic_workspace_size bytes."""
+    _bwd16("fa_bwd_deterministic", torch.bfloat16, q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal,
+           stream)
 
 
 def fa_bwd_f16(q, k, v, o, do, lse, dq, dk, dv, workspace, scale: float, causal: bool, stream=None) -> None:
@@ -156,10 +175,11 @@ def _bwd16(name, dtype, q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causa
 
 
 def fa_bwd_noalloc(q, k, v, o, do, lse, dq, dk, dv, scale: float, causal: bool, stream=None) -> None:
-    """Like fa_bwd but with no workspace: for callers that cannot allocate device
-    memory (they are handed only input and output buffers).  Uses the library's
-    fixed 8 MiB scratch array, so problems with B*H*ceil(N/128)*128 > 1,048,576
-    rows are rejected and calls that overlap on the GPU must not share it."""
+    """Like fa_bwd_deterministic (bf16, same results bit for bit) but with no workspace:
+    for callers that cannot allocate device memory (they are handed only input and
+    output buffers).  Uses the library's fixed 8 MiB scratch array, so problems with
+    B*H*ceil(N/128)*128 > 1,048,576 rows are rejected and calls that overlap on the GPU
+    must not share it."""
     B, H, N, D = q.shape
     for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", do), ("dq", dq), ("dk", dk), ("dv", dv)):
         _check(t, name, torch.bfloat16, (B, H, N, D))
@@ -206,6 +226,26 @@ def fa_bwd_dq(q, k, v, do, workspace, dq, scale: float, causal: bool, stream=Non
                                     B, H, N, D, float(scale), int(causal), _stream(stream)), "fa_bwd_dq")
 
 
+def fa_bwd_dkdvdq(q, k, v, do, workspace, dk, dv, scale: float, causal: bool, stream=None) -> None:
+    """Fused backward stage 2: dK, dV, and dQ added into the workspace's fp32 accumulator
+    (zeroed by fa_bwd_preprocess on a workspace of fa_bwd_workspace_size bytes)."""
+    B, H, N, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("do", do), ("dk", dk), ("dv", dv)):
+        _check(t, name, torch.bfloat16, (B, H, N, D))
+    wp, wn = _ws(workspace)
+    _raise(load_library().fa_bwd_dkdvdq(_p(q), _p(k), _p(v), _p(do), wp, wn, _p(dk), _p(dv),
+                                        B, H, N, D, float(scale), int(causal), _stream(stream)), "fa_bwd_dkdvdq")
+
+
+def fa_bwd_dq_finish(workspace, dq, scale: float, stream=None) -> None:
+    """Fused backward stage 3: dq <- scale * the workspace's fp32 dQ accumulator, as bf16."""
+    B, H, N, D = dq.shape
+    _check(dq, "dq", torch.bfloat16, (B, H, N, D))
+    wp, wn = _ws(workspace)
+    _raise(load_library().fa_bwd_dq_finish(wp, wn, _p(dq), B, H, N, D, float(scale), _stream(stream)),
+           "fa_bwd_dq_finish")
+
+
 def workspace_views(workspace, B: int, H: int, N: int):
     """(nl, delta) float32 views of a backward workspace, each (B, H, Npad)."""
     npad = (N + 127) // 128 * 128
@@ -238,14 +278,19 @@ def attention_forward(q, k, v, scale: float | None = None, causal: bool = False,
 
 
 def attention_backward(q, k, v, o, lse, do, scale: float | None = None, causal: bool = False, stream=None,
-                       workspace=None):
-    """Returns (dQ, dK, dV) for bf16 or fp16 inputs."""
+                       workspace=None, deterministic: bool = False):
+    """Returns (dQ, dK, dV) for bf16 or fp16 inputs (deterministic: bf16 only, the
+    bit-reproducible three-stage path)."""
     B, H, N, D = q.shape
     scale = default_scale(D) if scale is None else scale
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    size_fn = fa_bwd_deterministic_workspace_size if deterministic else fa_bwd_workspace_size
     if workspace is None:
-        workspace = torch.empty(fa_bwd_workspace_size(B, H, N, D), device=q.device, dtype=torch.uint8)
-    bwd = fa_bwd_f16 if q.dtype == torch.float16 else fa_bwd
+        workspace = torch.empty(size_fn(B, H, N, D), device=q.device, dtype=torch.uint8)
+    if deterministic:
+        bwd = fa_bwd_deterministic
+    else:
+        bwd = fa_bwd_f16 if q.dtype == torch.float16 else fa_bwd
     bwd(q, k, v, o, do, lse, dq, dk, dv, workspace, scale, causal, stream)
     return dq, dk, dv
 
@@ -306,28 +351,35 @@ def attention_fwd_bwd_from_host(q_h, k_h, v_h, do_h, scale: float, causal: bool,
 
 
 class HostStepPipeline:
-    """Forward + backward steps whose inputs and results live in pinned host memory,
-    pipelined over `depth` sets of device buffers and three CUDA streams: the upload of
-    step i+1 and the download of step i-1 run on the copy engines while step i computes.
+    """Attention steps whose inputs and results live in pinned host memory, pipelined over
+    `depth` sets of device buffers and three CUDA streams: the upload of step i+1 and the
+    download of step i-1 run on the copy engines while step i computes.
 
-    submit(q, k, v, do, out, scale, causal) queues one step: copy q, k, v, dO (pinned
-    host tensors of shape (B,H,N,D)) to the device, fa_fwd + fa_bwd (or the fp16 entry
-    points) on the compute stream, then copy O, lse, dQ, dK, dV into `out` (a dict of
-    pinned host tensors, as returned by host_outputs()).  Results of a step are in `out`
-    once wait() (or synchronize()) has returned; a caller keeping several steps in flight
-    gives each its own `out`.  The library's own kernels do all the arithmetic; this class
-    only orders copies and launches."""
+    submit(q, k, v, do, out, scale, causal) queues one step: copy q, k, v (and dO when
+    `backward`) from pinned host tensors of shape (B,H,N,D) to the device, run the forward
+    (fa_fwd, fa_fwd_f16 or fa_fwd_f32 by dtype) and, when `backward`, fa_bwd / fa_bwd_f16
+    on the compute stream, then copy O, lse (and dQ, dK, dV) into `out` (a dict of pinned
+    host tensors, as returned by host_outputs()).  Results of a step are in `out` once
+    synchronize() has returned; a caller keeping several steps in flight gives each its
+    own `out`.  The library's own kernels do all the arithmetic; this class only orders
+    copies and launches."""
 
-    def __init__(self, B: int, H: int, N: int, D: int, dtype=torch.bfloat16, depth: int = 2, device=None):
+    def __init__(self, B: int, H: int, N: int, D: int, dtype=torch.bfloat16, depth: int = 2, device=None,
+                 backward: bool = True):
+        if backward and dtype == torch.float32:
+            raise ValueError("the fp32 path has no backward")
         dev = torch.device("cuda") if device is None else torch.device(device)
-        self.shape, self.dtype, self.depth = (B, H, N, D), dtype, depth
+        self.shape, self.dtype, self.depth, self.backward = (B, H, N, D), dtype, depth, backward
+        self.inputs = ("q", "k", "v", "do") if backward else ("q", "k", "v")
+        self.outputs = ("o", "lse", "dq", "dk", "dv") if backward else ("o", "lse")
         self.bufs = []
         for _ in range(depth):
             b = {n: torch.empty(B, H, N, D, device=dev, dtype=dtype)
-                 for n in ("q", "k", "v", "do", "o", "dq", "dk", "dv")}
+                 for n in self.inputs + tuple(n for n in self.outputs if n != "lse")}
             b["lse"] = torch.empty(B, H, N, device=dev, dtype=torch.float32)
             self.bufs.append(b)
-        self.ws = torch.empty(fa_bwd_workspace_size(B, H, N, D), device=dev, dtype=torch.uint8)
+        self.ws = (torch.empty(fa_bwd_workspace_size(B, H, N, D), device=dev, dtype=torch.uint8)
+                   if backward else None)
         self.s_h2d, self.s_comp, self.s_d2h = (torch.cuda.Stream(dev) for _ in range(3))
         self.ev_loaded = [torch.cuda.Event() for _ in range(depth)]    # inputs of the slot on the device
         self.ev_computed = [torch.cuda.Event() for _ in range(depth)]  # slot's kernels done
@@ -337,37 +389,41 @@ class HostStepPipeline:
 
     def host_outputs(self):
         B, H, N, D = self.shape
-        out = {n: torch.empty(B, H, N, D, dtype=self.dtype).pin_memory() for n in ("o", "dq", "dk", "dv")}
+        out = {n: torch.empty(B, H, N, D, dtype=self.dtype).pin_memory() for n in self.outputs if n != "lse"}
         out["lse"] = torch.empty(B, H, N, dtype=torch.float32).pin_memory()
         return out
 
     def submit(self, q_h, k_h, v_h, do_h, out, scale: float, causal: bool):
-        """Queues one step; returns (h2d_bytes, d2h_bytes) of its copies."""
+        """Queues one step (do_h is ignored without `backward`); returns (h2d_bytes, d2h_bytes)
+        of its copies."""
         s = self.i % self.depth
         b = self.bufs[s]
+        hosts = (q_h, k_h, v_h, do_h)[: len(self.inputs)]
         if self.used[s]:
             self.s_h2d.wait_event(self.ev_computed[s])     # the kernels of step i-depth read these inputs
         with torch.cuda.stream(self.s_h2d):
-            for n, h in (("q", q_h), ("k", k_h), ("v", v_h), ("do", do_h)):
+            for n, h in zip(self.inputs, hosts):
                 b[n].copy_(h, non_blocking=True)
         self.ev_loaded[s].record(self.s_h2d)
         self.s_comp.wait_event(self.ev_loaded[s])
         if self.used[s]:
             self.s_comp.wait_event(self.ev_fetched[s])     # step i-depth's results have left these buffers
-        fwd, bwd = (fa_fwd_f16, fa_bwd_f16) if self.dtype == torch.float16 else (fa_fwd, fa_bwd)
+        fwd = {torch.float16: fa_fwd_f16, torch.float32: fa_fwd_f32}.get(self.dtype, fa_fwd)
         fwd(b["q"], b["k"], b["v"], b["o"], b["lse"], scale, causal, self.s_comp)
-        bwd(b["q"], b["k"], b["v"], b["o"], b["do"], b["lse"], b["dq"], b["dk"], b["dv"], self.ws, scale, causal,
-            self.s_comp)
+        if self.backward:
+            bwd = fa_bwd_f16 if self.dtype == torch.float16 else fa_bwd
+            bwd(b["q"], b["k"], b["v"], b["o"], b["do"], b["lse"], b["dq"], b["dk"], b["dv"], self.ws, scale, causal,
+                self.s_comp)
         self.ev_computed[s].record(self.s_comp)
         self.s_d2h.wait_event(self.ev_computed[s])
         with torch.cuda.stream(self.s_d2h):
-            for n in ("o", "lse", "dq", "dk", "dv"):
+            for n in self.outputs:
                 out[n].copy_(b[n], non_blocking=True)
         self.ev_fetched[s].record(self.s_d2h)
         self.used[s] = True
         self.i += 1
-        h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, do_h))
-        d2h = sum(out[n].numel() * out[n].element_size() for n in ("o", "lse", "dq", "dk", "dv"))
+        h2d = sum(t.numel() * t.element_size() for t in hosts)
+        d2h = sum(out[n].numel() * out[n].element_size() for n in self.outputs)
         return h2d, d2h
 
     def synchronize(self):

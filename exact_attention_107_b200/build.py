@@ -22,7 +22,7 @@ INCLUDE = ROOT / "include"
 BUILD = PKG / "_build"
 LIB = PKG / "libfa.so"
 SOURCES = ["fa_api.cu", "fa_fwd_sm100.cu", "fa_fwd_d256_sm100.cu", "fa_fwd_f32.cu", "fa_bwd_sm100.cu",
-           "fa_bwd_d256_sm100.cu", "fa_noalloc.cu"]
+           "fa_bwd_d256_sm100.cu", "fa_bwd_fused_sm100.cu", "fa_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
           "-I" + str(INCLUDE), "-I" + str(CSRC)]

@@ -99,11 +99,31 @@ int launch_status(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_LAUN
 
 bool scale_ok(float scale) { return std::isfinite(scale) && scale > 0.f; }
 
+// Columns of the 16-bit kernels' tiles for head dim D (the fused backward's dQ accumulator
+// holds this many floats per row); 0 for D = 256, which has no fused backward.
+int tile_cols(int D) { return D <= 64 ? 64 : (D <= 128 ? 128 : 0); }
+
+// Bytes of the backward's row statistics: -lse*log2(e) and delta for B*H*Npad rows.
+size_t stats_bytes(int B, int H, int N) {
+  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  return 2 * static_cast<size_t>(B) * H * npad * sizeof(float);
+}
+
+// Heads per L2 group of the grouped CTA order: as many heads as fit their shared data
+// (bytes_per_head) into 64 MiB, about half of the B200's 126 MB L2.
+int heads_per_group(long long bytes_per_head, int BH) {
+  const long long budget = 64LL << 20;
+  long long hg = bytes_per_head > 0 ? budget / bytes_per_head : BH;
+  if (hg < 1) hg = 1;
+  if (hg > BH) hg = BH;
+  return static_cast<int>(hg);
+}
+
 }  // namespace
 
 extern "C" {
 
-int fa_version(void) { return 10000; }
+int fa_version(void) { return 20000; }
 
 const char* fa_status_string(int status) {
   switch (status) {
@@ -164,6 +184,8 @@ static int fwd16(const void* q, const void* k, const void* v, void* o, float* ls
   a.causal = causal;
   a.status = ds->status;
   a.num_sms = ds->num_sms;
+  // The forward's CTAs of one head share that head's K and V tiles.
+  a.hg = heads_per_group(4LL * N * D, BH);
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   return launch_status(D == 256 ? fa::launch_fwd_d256(a, s) : fa::launch_fwd_16(a, s));
 }
@@ -197,29 +219,35 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
 size_t fa_bwd_workspace_size(int B, int H, int N, int D) {
   if (check_shape(B, H, N, D, true, true) != FA_OK) return 0;
   const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
-  return 2 * static_cast<size_t>(B) * H * npad * sizeof(float);    // a multiple of 1024 bytes
-}
-
-// Workspace views: ws_nl = [0, B*H*Npad) floats, ws_delta = [B*H*Npad, 2*B*H*Npad).
-static int workspace_views(void* ws, size_t ws_bytes, int B, int H, int N, int D, fa::BwdLaunch* a) {
-  if (!ws || ws_bytes < fa_bwd_workspace_size(B, H, N, D)) return FA_ERR_WORKSPACE;
-  if (!aligned16(ws)) return FA_ERR_ALIGN;
-  a->Npad = (N + 127) / 128 * 128;
-  a->ws_nl = static_cast<float*>(ws);
-  a->ws_delta = a->ws_nl + static_cast<size_t>(B) * H * a->Npad;
-  return FA_OK;
+  const size_t rows = static_cast<size_t>(B) * H * npad;
+  return rows * (2 + static_cast<size_t>(tile_cols(D))) * sizeof(float);   // a multiple of 1024 bytes
 }
 
 }  // extern "C"
 
+// Workspace views: ws_nl = [0, R) floats, ws_delta = [R, 2R) with R = B*H*Npad, and (with_acc,
+// head dims up to 128) the fused path's dQ accumulator ws_dq = [2R, 2R + R*DK).
+static int workspace_views(void* ws, size_t ws_bytes, int B, int H, int N, int D, bool with_acc, fa::BwdLaunch* a) {
+  const size_t need = with_acc ? fa_bwd_workspace_size(B, H, N, D) : stats_bytes(B, H, N);
+  if (!ws || ws_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return FA_ERR_ALIGN;
+  a->Npad = (N + 127) / 128 * 128;
+  const size_t rows = static_cast<size_t>(B) * H * a->Npad;
+  a->ws_nl = static_cast<float*>(ws);
+  a->ws_delta = a->ws_nl + rows;
+  a->DK = tile_cols(D);
+  a->ws_dq = (with_acc && a->DK > 0) ? a->ws_delta + rows : nullptr;
+  return FA_OK;
+}
+
 static int preprocess16(const void* o, const void* dO, const float* lse, void* workspace, size_t workspace_bytes,
-                        int B, int H, int N, int D, void* stream, bool f16) {
+                        int B, int H, int N, int D, bool with_acc, void* stream, bool f16) {
   if (!o || !dO || !lse) return FA_ERR_NULL;
   int st = check_shape(B, H, N, D, true, true);
   if (st != FA_OK) return st;
   if (!aligned16(o) || !aligned16(dO) || !aligned16(lse)) return FA_ERR_ALIGN;
   fa::BwdLaunch a{};
-  if ((st = workspace_views(workspace, workspace_bytes, B, H, N, D, &a)) != FA_OK) return st;
+  if ((st = workspace_views(workspace, workspace_bytes, B, H, N, D, with_acc, &a)) != FA_OK) return st;
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
   a.f16 = f16 ? 1 : 0;
@@ -233,21 +261,22 @@ static int preprocess16(const void* o, const void* dO, const float* lse, void* w
 }
 
 static int bwd_common(const void* q, const void* k, const void* v, const void* dO, const void* workspace,
-                      size_t workspace_bytes, int B, int H, int N, int D, float scale, int causal, int q_box_rows,
+                      size_t workspace_bytes, int B, int H, int N, int D, float scale, int causal, bool with_acc,
                       bool f16, fa::BwdLaunch* a) {
   if (!q || !k || !v || !dO) return FA_ERR_NULL;
   int st = check_shape(B, H, N, D, true, true);
   if (st != FA_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO)) return FA_ERR_ALIGN;
-  if ((st = workspace_views(const_cast<void*>(workspace), workspace_bytes, B, H, N, D, a)) != FA_OK) return st;
+  if ((st = workspace_views(const_cast<void*>(workspace), workspace_bytes, B, H, N, D, with_acc, a)) != FA_OK)
+    return st;
   if (!scale_ok(scale) || (causal != 0 && causal != 1)) return FA_ERR_ARG;
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
   const int BH = B * H;
-  if ((st = make_tmap(&a->tmQ, q, BH, N, D, q_box_rows, f16)) != FA_OK) return st;
+  if ((st = make_tmap(&a->tmQ, q, BH, N, D, 128, f16)) != FA_OK) return st;
   if ((st = make_tmap(&a->tmK, k, BH, N, D, 128, f16)) != FA_OK) return st;
   if ((st = make_tmap(&a->tmV, v, BH, N, D, 128, f16)) != FA_OK) return st;
-  if ((st = make_tmap(&a->tmdO, dO, BH, N, D, q_box_rows, f16)) != FA_OK) return st;
+  if ((st = make_tmap(&a->tmdO, dO, BH, N, D, 128, f16)) != FA_OK) return st;
   a->f16 = f16 ? 1 : 0;
   a->BH = BH;
   a->N = N;
@@ -256,6 +285,8 @@ static int bwd_common(const void* q, const void* k, const void* v, const void* d
   a->causal = causal;
   a->status = ds->status;
   a->num_sms = ds->num_sms;
+  // The fused kernel's CTAs of one head share that head's Q and dO tiles and dQ accumulator.
+  a->hg = heads_per_group(static_cast<long long>(a->Npad) * (4LL * D + 4LL * a->DK), BH);
   return FA_OK;
 }
 
@@ -265,7 +296,7 @@ static int dkdv16(const void* q, const void* k, const void* v, const void* dO, c
   if (!dk || !dv) return FA_ERR_NULL;
   if (!aligned16(dk) || !aligned16(dv)) return FA_ERR_ALIGN;
   fa::BwdLaunch a{};
-  int st = bwd_common(q, k, v, dO, workspace, workspace_bytes, B, H, N, D, scale, causal, 128, f16, &a);
+  int st = bwd_common(q, k, v, dO, workspace, workspace_bytes, B, H, N, D, scale, causal, false, f16, &a);
   if (st != FA_OK) return st;
   if ((st = make_tmap(&a.tmdK, dk, a.BH, N, D, 32, f16)) != FA_OK) return st;
   if ((st = make_tmap(&a.tmdV, dv, a.BH, N, D, 32, f16)) != FA_OK) return st;
@@ -278,36 +309,108 @@ static int dq16(const void* q, const void* k, const void* v, const void* dO, con
   if (!dq) return FA_ERR_NULL;
   if (!aligned16(dq)) return FA_ERR_ALIGN;
   fa::BwdLaunch a{};
-  int st = bwd_common(q, k, v, dO, workspace, workspace_bytes, B, H, N, D, scale, causal, 128, f16, &a);
+  int st = bwd_common(q, k, v, dO, workspace, workspace_bytes, B, H, N, D, scale, causal, false, f16, &a);
   if (st != FA_OK) return st;
   if ((st = make_tmap(&a.tmdQ, dq, a.BH, N, D, 32, f16)) != FA_OK) return st;
   return launch_status(fa::launch_bwd_dq(a, static_cast<cudaStream_t>(stream)));
 }
 
-static int bwd16(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
-                 void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int D,
-                 float scale, int causal, void* stream, bool f16) {
+static int dkdvdq16(const void* q, const void* k, const void* v, const void* dO, void* workspace,
+                    size_t workspace_bytes, void* dk, void* dv, int B, int H, int N, int D, float scale, int causal,
+                    void* stream, bool f16) {
+  if (!dk || !dv) return FA_ERR_NULL;
+  if (!aligned16(dk) || !aligned16(dv)) return FA_ERR_ALIGN;
+  if (D > 128) return check_shape(B, H, N, D, true, false);     // no fused kernel for D = 256
+  fa::BwdLaunch a{};
+  int st = bwd_common(q, k, v, dO, workspace, workspace_bytes, B, H, N, D, scale, causal, true, f16, &a);
+  if (st != FA_OK) return st;
+  if ((st = make_tmap(&a.tmdK, dk, a.BH, N, D, 32, f16)) != FA_OK) return st;
+  if ((st = make_tmap(&a.tmdV, dv, a.BH, N, D, 32, f16)) != FA_OK) return st;
+  return launch_status(fa::launch_bwd_fused(a, static_cast<cudaStream_t>(stream)));
+}
+
+static int dq_finish16(const void* workspace, size_t workspace_bytes, void* dq, int B, int H, int N, int D,
+                       float scale, void* stream, bool f16) {
+  if (!dq) return FA_ERR_NULL;
+  int st = check_shape(B, H, N, D, true, false);
+  if (st != FA_OK) return st;
+  if (!aligned16(dq)) return FA_ERR_ALIGN;
+  if (!scale_ok(scale)) return FA_ERR_ARG;
+  fa::BwdLaunch a{};
+  if ((st = workspace_views(const_cast<void*>(workspace), workspace_bytes, B, H, N, D, true, &a)) != FA_OK) return st;
+  DeviceState* ds = nullptr;
+  if ((st = device_state(&ds)) != FA_OK) return st;
+  a.f16 = f16 ? 1 : 0;
+  a.BH = B * H;
+  a.N = N;
+  a.D = D;
+  a.scale = scale;
+  return launch_status(fa::launch_bwd_dq_finish(a, dq, static_cast<cudaStream_t>(stream)));
+}
+
+// Validation shared by the two complete backward entry points, so that an error launches nothing.
+static int bwd_validate(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                        void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, size_t ws_need,
+                        int B, int H, int N, int D, float scale, int causal) {
   if (!q || !k || !v || !o || !dO || !lse || !dq || !dk || !dv) return FA_ERR_NULL;
   int st = check_shape(B, H, N, D, true, true);
   if (st != FA_OK) return st;
-  if (!workspace || workspace_bytes < fa_bwd_workspace_size(B, H, N, D)) return FA_ERR_WORKSPACE;
-  // Validate everything the three stages will check, so that an error launches nothing.
+  if (!workspace || workspace_bytes < ws_need) return FA_ERR_WORKSPACE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dO) || !aligned16(lse) ||
       !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
     return FA_ERR_ALIGN;
   if (!scale_ok(scale) || (causal != 0 && causal != 1)) return FA_ERR_ARG;
-  if ((st = preprocess16(o, dO, lse, workspace, workspace_bytes, B, H, N, D, stream, f16)) != FA_OK) return st;
-  if ((st = dkdv16(q, k, v, dO, workspace, workspace_bytes, dk, dv, B, H, N, D, scale, causal, stream, f16)) !=
+  return FA_OK;
+}
+
+// fa_bwd / fa_bwd_f16: the fused kernel for head dims up to 128 (preprocess, which also
+// zeroes the dQ accumulator; dK/dV/dQ kernel; dQ finish), the two-CTA three-stage path at 256.
+static int bwd16(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                 void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int D,
+                 float scale, int causal, void* stream, bool f16) {
+  int st = bwd_validate(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes,
+                        fa_bwd_workspace_size(B, H, N, D), B, H, N, D, scale, causal);
+  if (st != FA_OK) return st;
+  const bool fused = tile_cols(D) > 0;
+  if ((st = preprocess16(o, dO, lse, workspace, workspace_bytes, B, H, N, D, fused, stream, f16)) != FA_OK) return st;
+  if (!fused) {
+    if ((st = dkdv16(q, k, v, dO, workspace, workspace_bytes, dk, dv, B, H, N, D, scale, causal, stream, f16)) !=
+        FA_OK)
+      return st;
+    return dq16(q, k, v, dO, workspace, workspace_bytes, dq, B, H, N, D, scale, causal, stream, f16);
+  }
+  if ((st = dkdvdq16(q, k, v, dO, workspace, workspace_bytes, dk, dv, B, H, N, D, scale, causal, stream, f16)) !=
       FA_OK)
+    return st;
+  return dq_finish16(workspace, workspace_bytes, dq, B, H, N, D, scale, stream, f16);
+}
+
+// fa_bwd_deterministic: preprocess, the dK/dV kernel and the dQ kernel (no atomics).
+static int bwd_det16(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse,
+                     void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N,
+                     int D, float scale, int causal, void* stream, bool f16) {
+  int st = bwd_validate(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, stats_bytes(B, H, N), B, H, N,
+                        D, scale, causal);
+  if (st != FA_OK) return st;
+  if ((st = preprocess16(o, dO, lse, workspace, workspace_bytes, B, H, N, D, false, stream, f16)) != FA_OK) return st;
+  if ((st = dkdv16(q, k, v, dO, workspace, workspace_bytes, dk, dv, B, H, N, D, scale, causal, stream, f16)) != FA_OK)
     return st;
   return dq16(q, k, v, dO, workspace, workspace_bytes, dq, B, H, N, D, scale, causal, stream, f16);
 }
 
 extern "C" {
 
+size_t fa_bwd_deterministic_workspace_size(int B, int H, int N, int D) {
+  if (check_shape(B, H, N, D, true, true) != FA_OK) return 0;
+  return stats_bytes(B, H, N);
+}
+
 int fa_bwd_preprocess(const void* o, const void* dO, const float* lse, void* workspace, size_t workspace_bytes,
                       int B, int H, int N, int D, void* stream) {
-  return preprocess16(o, dO, lse, workspace, workspace_bytes, B, H, N, D, stream, false);
+  // The dQ accumulator is zeroed when the workspace holds one (fa_bwd_workspace_size bytes).
+  const size_t full = fa_bwd_workspace_size(B, H, N, D);
+  const bool with_acc = tile_cols(D) > 0 && full > 0 && workspace_bytes >= full;
+  return preprocess16(o, dO, lse, workspace, workspace_bytes, B, H, N, D, with_acc, stream, false);
 }
 
 int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO, const void* workspace,
@@ -321,6 +424,17 @@ int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO, const
   return dq16(q, k, v, dO, workspace, workspace_bytes, dq, B, H, N, D, scale, causal, stream, false);
 }
 
+int fa_bwd_dkdvdq(const void* q, const void* k, const void* v, const void* dO, void* workspace,
+                  size_t workspace_bytes, void* dk, void* dv, int B, int H, int N, int D, float scale, int causal,
+                  void* stream) {
+  return dkdvdq16(q, k, v, dO, workspace, workspace_bytes, dk, dv, B, H, N, D, scale, causal, stream, false);
+}
+
+int fa_bwd_dq_finish(const void* workspace, size_t workspace_bytes, void* dq, int B, int H, int N, int D, float scale,
+                     void* stream) {
+  return dq_finish16(workspace, workspace_bytes, dq, B, H, N, D, scale, stream, false);
+}
+
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO, const float* lse, void* dq,
            void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int D, float scale,
            int causal, void* stream) {
@@ -331,6 +445,13 @@ int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o, const
                void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N, int D,
                float scale, int causal, void* stream) {
   return bwd16(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N, D, scale, causal, stream, true);
+}
+
+int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                         int B, int H, int N, int D, float scale, int causal, void* stream) {
+  return bwd_det16(q, k, v, o, dO, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N, D, scale, causal, stream,
+                   false);
 }
 
 }  // extern "C"

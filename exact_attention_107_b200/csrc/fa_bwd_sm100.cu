@@ -44,7 +44,8 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint16_t* __r
                                                              const uint16_t* __restrict__ dO,
                                                              const float* __restrict__ lse,
                                                              float* __restrict__ ws_nl, float* __restrict__ ws_delta,
-                                                             int N, int Npad, int D, long long padded_rows) {
+                                                             float* __restrict__ ws_dq, int N, int Npad, int D, int DK,
+                                                             long long padded_rows) {
   const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long prow = gt / kLanesPerRow;          // row in the padded (B*H, Npad) layout
   const int part = static_cast<int>(gt % kLanesPerRow);
@@ -68,6 +69,14 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint16_t* __r
   if (prow < padded_rows && part == 0) {
     ws_delta[prow] = acc;
     ws_nl[prow] = real ? -lse[row] * kLog2e : -CUDART_INF_F;
+  }
+  // The fused backward adds dQ into an fp32 accumulator of DK floats per padded row: zero
+  // this row's share of it (the accumulator's tile layout keeps a row's DK floats
+  // contiguous only per tile, but zeroing [prow * DK, prow * DK + DK) over all rows covers it).
+  if (ws_dq != nullptr && prow < padded_rows) {
+    const int per_lane = DK / kLanesPerRow;             // 8 or 16 floats
+    float4* z = reinterpret_cast<float4*>(ws_dq + prow * DK + part * per_lane);
+    for (int i = 0; i < per_lane / 4; ++i) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
@@ -686,7 +695,7 @@ cudaError_t preprocess_impl(const BwdLaunch& a, cudaStream_t stream) {
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   bwd_preprocess_kernel<kLanesPerRow, F16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
       static_cast<const uint16_t*>(a.o), static_cast<const uint16_t*>(a.dO), a.lse, a.ws_nl, a.ws_delta,
-      a.N, a.Npad, a.D, padded_rows);
+      a.ws_dq, a.N, a.Npad, a.D, a.DK, padded_rows);
   return cudaGetLastError();
 }
 

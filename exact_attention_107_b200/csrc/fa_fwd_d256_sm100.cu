@@ -66,7 +66,7 @@ template <bool CAUSAL, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_d256_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                    float* __restrict__ lse, int N, int BH, int nqt, float scale_log2, int* status) {
+                    float* __restrict__ lse, int N, int BH, int nqt, int hg, float scale_log2, int* status) {
   using L = Smem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -80,12 +80,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Work item: one 128-row query tile of one (batch, head); causal work grows with the
   // query index, so the heaviest tiles are handed out first.
   int qt, bh;
-  if (CAUSAL) {
-    qt = nqt - 1 - static_cast<int>(blockIdx.x / BH);
-    bh = blockIdx.x % BH;
-  } else {
-    qt = blockIdx.x % nqt;
-    bh = blockIdx.x / nqt;
+  {
+    const WorkItem wi = grouped_order(static_cast<int>(blockIdx.x), BH, nqt, hg);
+    bh = wi.bh;
+    qt = CAUSAL ? nqt - 1 - wi.tile : wi.tile;
   }
   const int q0 = qt * kBM;
   const int nkv_all = (N + kBN - 1) / kBN;
@@ -342,7 +340,7 @@ cudaError_t launch_impl(const FwdLaunch& a, cudaStream_t stream) {
   const int nqt = (a.N + kBM - 1) / kBM;
   const unsigned grid = static_cast<unsigned>(nqt) * static_cast<unsigned>(a.BH);
   const float scale_log2 = a.scale * 1.44269504088896340736f;
-  kern<<<grid, kThreads, Smem::kBytes, stream>>>(a.tmQ, a.tmK, a.tmV, a.tmO, a.lse, a.N, a.BH, nqt, scale_log2,
+  kern<<<grid, kThreads, Smem::kBytes, stream>>>(a.tmQ, a.tmK, a.tmV, a.tmO, a.lse, a.N, a.BH, nqt, a.hg, scale_log2,
                                                    a.status);
   return cudaGetLastError();
 }

@@ -82,7 +82,7 @@ template <int D, bool CAUSAL, bool F16>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                    float* __restrict__ lse, int N, int BH, int nqb, float scale_log2, int* status) {
+                    float* __restrict__ lse, int N, int BH, int nqb, int hg, float scale_log2, int* status) {
   using L = FwdSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -96,12 +96,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Work item: 256 query rows (two tiles) of one (batch, head).  Causal work grows
   // with the query index, so the heaviest blocks are handed out first.
   int qblk, bh;
-  if (CAUSAL) {
-    qblk = nqb - 1 - static_cast<int>(blockIdx.x / BH);
-    bh = blockIdx.x % BH;
-  } else {
-    qblk = blockIdx.x % nqb;
-    bh = blockIdx.x / nqb;
+  {
+    const WorkItem wi = grouped_order(static_cast<int>(blockIdx.x), BH, nqb, hg);
+    bh = wi.bh;
+    qblk = CAUSAL ? nqb - 1 - wi.tile : wi.tile;
   }
   const int nkv_all = (N + kBN - 1) / kBN;
   int q0[2], nkv[2];
@@ -397,7 +395,7 @@ cudaError_t launch_impl(const FwdLaunch& a, cudaStream_t stream) {
   const int nqb = (a.N + 2 * kBM - 1) / (2 * kBM);
   const unsigned grid = static_cast<unsigned>(nqb) * static_cast<unsigned>(a.BH);
   const float scale_log2 = a.scale * 1.44269504088896340736f;
-  kern<<<grid, kThreads, L::kBytes, stream>>>(a.tmQ, a.tmK, a.tmV, a.tmO, a.lse, a.N, a.BH, nqb, scale_log2,
+  kern<<<grid, kThreads, L::kBytes, stream>>>(a.tmQ, a.tmK, a.tmV, a.tmO, a.lse, a.N, a.BH, nqb, a.hg, scale_log2,
                                                a.status);
   return cudaGetLastError();
 }

@@ -6,7 +6,24 @@
 
 namespace fa {
 
+constexpr int kStatusLaunch = 6;   // FA_ERR_LAUNCH (a kernel found its launch unusable)
 constexpr int kStatusTimeout = 7;  // FA_ERR_TIMEOUT
+
+// Order of the CTAs of a (head, tile) grid.  Heads are taken in groups of `hg` whose
+// data fits in L2 together; inside a group the order is tile-major (tile 0 of every
+// head of the group first, then tile 1, ...), so that with causal masking the heaviest
+// tiles of a group start first, and CTAs that run at the same time share their heads'
+// K/V (forward) or Q/dO/dQ (backward) through L2 instead of re-reading device memory.
+struct WorkItem {
+  int bh, tile;
+};
+__host__ __device__ inline WorkItem grouped_order(int cta, int BH, int ntiles, int hg) {
+  const long long per_group = static_cast<long long>(hg) * ntiles;
+  const int g = static_cast<int>(cta / per_group);
+  const int local = static_cast<int>(cta - g * per_group);
+  const int gh = (BH - g * hg) < hg ? (BH - g * hg) : hg;     // the last group may be smaller
+  return {g * hg + local % gh, local / gh};
+}
 
 // bf16 / fp16 forward (fa_fwd_sm100.cu).  Tensor maps are 3-D (D, N, B*H) of the
 // element type with 64 x 128 x 1 boxes (O: 64 x 32 x 1) and 128-byte swizzle.
@@ -17,6 +34,7 @@ struct FwdLaunch {
   float scale;
   int causal;
   int f16;           // element type: 0 = bf16, 1 = fp16
+  int hg;            // heads per L2 group (grouped_order)
   int* status;
   int num_sms;
 };
@@ -39,7 +57,10 @@ struct BwdLaunch {
   const float* lse;
   float* ws_nl;
   float* ws_delta;
+  float* ws_dq;      // fp32 dQ accumulator of the fused path (B*H*Npad*DK floats), or null
   int BH, N, Npad, D;
+  int DK;            // columns of the kernels' tiles: 64 (D <= 64) or 128 (D in {96, 128})
+  int hg;            // heads per L2 group (grouped_order)
   float scale;
   int causal;
   int f16;           // element type of q, k, v, o, dO and the gradients: 0 = bf16, 1 = fp16
@@ -49,6 +70,10 @@ struct BwdLaunch {
 cudaError_t launch_bwd_preprocess(const BwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_bwd_dkdv(const BwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_bwd_dq(const BwdLaunch& a, cudaStream_t stream);
+// Fused backward (fa_bwd_fused_sm100.cu), DK in {64, 128}: dK, dV written, dQ added into
+// ws_dq (which the preprocess kernel zeroed); then dq_finish writes scale * ws_dq to dq.
+cudaError_t launch_bwd_fused(const BwdLaunch& a, cudaStream_t stream);
+cudaError_t launch_bwd_dq_finish(const BwdLaunch& a, void* dq, cudaStream_t stream);
 // Head dimension 256 (fa_bwd_d256_sm100.cu): two CTAs per tile, one per half of D.
 cudaError_t launch_bwd_dkdv_d256(const BwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_bwd_dq_d256(const BwdLaunch& a, cudaStream_t stream);

@@ -2,8 +2,8 @@
 
 Method: Cody-Waite style range reduction (W. J. Cody and W. Waite, "Software
 Manual for the Elementary Functions", 1980): 2^x = 2^n * 2^f with n = round(x)
-and f = x - n in [-1/2, 1/2]; 2^n is applied by adding n to the float's exponent
-field.  2^f is approximated by the cubic p(f) = c0 + c1 f + c2 f^2 + c3 f^3
+and f = x - n in [-1/2, 1/2]; 2^n is built as a float from its exponent field and
+applied by one multiplication.  2^f is approximated by the cubic p(f) = c0 + c1 f + c2 f^2 + c3 f^3
 whose maximum *relative* error on [-1/2, 1/2] is minimised with the Remez
 exchange algorithm (E. Ya. Remez, 1934) on the weighted Haar system
 {1, f, f^2, f^3} * 2^-f.  (Pinning c0 = 1 would make every basis function but
@@ -52,10 +52,11 @@ def remez_relative(degree: int, iters: int = 50):
 
 
 def eval_f32(x: np.ndarray, c: np.ndarray) -> np.ndarray:
-    """The kernels' steps in float32: clamp, round-to-integer by the 1.5*2^23 trick,
-    f = x - n, Horner polynomial, exponent add."""
-    x = np.maximum(x.astype(np.float32), np.float32(-125.0))
-    magic = np.float32(12582912.0)
+    """The kernels' steps in float32: NaN-keeping clamp, round-to-integer by adding
+    1.5*2^23 + 127 (the sum's low 9 mantissa bits are then n + 127), f = x - n, Horner
+    polynomial, times 2^n made from those bits as an exponent field."""
+    x = np.maximum(x.astype(np.float32), np.float32(-125.0))      # numpy's maximum keeps NaN
+    magic = np.float32(12583039.0)
     t = (x + magic).astype(np.float32)
     n = (t - magic).astype(np.float32)
     f = (x - n).astype(np.float32)
@@ -63,8 +64,9 @@ def eval_f32(x: np.ndarray, c: np.ndarray) -> np.ndarray:
     p = c[3] * f + c[2]
     p = p.astype(np.float32) * f + c[1]
     p = p.astype(np.float32) * f + c[0]
-    bits = p.astype(np.float32).view(np.int32) + (t.view(np.int32) << 23)
-    return bits.astype(np.int32).view(np.float32)
+    scale = (t.view(np.int32) << 23).astype(np.int32).view(np.float32)
+    with np.errstate(invalid="ignore", over="ignore"):
+        return (p.astype(np.float32) * scale).astype(np.float32)
 
 
 if __name__ == "__main__":

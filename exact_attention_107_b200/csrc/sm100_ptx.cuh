@@ -184,6 +184,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -241,28 +250,38 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Maximum that propagates NaN (max.NaN.f32): max(NaN, y) is NaN, max(-inf, y) is y.
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
 // 2^x for two values at once on the FMA pipe (packed fp32x2 arithmetic), so that part
 // of the exponentials can bypass the MUFU unit.  Cody-Waite range reduction
-// (x = n + f, n = round(x) via the 1.5*2^23 rounding trick, f in [-1/2, 1/2]), a cubic
-// for 2^f whose coefficients minimise the maximum relative error on [-1/2, 1/2]
-// (Remez exchange; derived by gen_exp2_poly.py in this directory), and 2^n applied
-// by adding n to the exponent field.  Max relative error 7.8e-5 for x in [-125, 10];
-// x below -125 (including -inf) is clamped to -125, i.e. a result of ~2.4e-38.
+// (x = n + f, n = round(x) by adding 1.5*2^23 + 127 so that the sum's low mantissa
+// bits hold n + 127, f in [-1/2, 1/2]), a cubic for 2^f whose coefficients minimise
+// the maximum relative error on [-1/2, 1/2] (Remez exchange; derived by
+// gen_exp2_poly.py in this directory), and 2^n, built from those low bits as a
+// float's exponent field, applied by one multiplication.  Max relative error 7.8e-5
+// for x in [-125, 10]; x below -125 (including -inf) is clamped to -125, i.e. a
+// result of ~2.4e-38.  NaN propagates as it does through MUFU ex2: the clamp keeps a
+// NaN, the polynomial of a NaN is NaN, and NaN times the scale is NaN.
 constexpr float kExp2C0 = 0.99992805719375610f;   // 0x3f7ffb49
 constexpr float kExp2C1 = 0.69326096773147583f;   // 0x3f31798d
 constexpr float kExp2C2 = 0.24261112511157990f;   // 0x3e786f0d
 constexpr float kExp2C3 = 0.05517166852951050f;   // 0x3d61fbb0
+constexpr float kExp2Round = 12583039.f;          // 1.5 * 2^23 + 127
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = __fadd2_rn(x, make_float2(12582912.f, 12582912.f));
-  const float2 n = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  x.x = fmax_nan(x.x, -125.f);
+  x.y = fmax_nan(x.y, -125.f);
+  const float2 t = __fadd2_rn(x, make_float2(kExp2Round, kExp2Round));
+  const float2 n = __fadd2_rn(t, make_float2(-kExp2Round, -kExp2Round));
   const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
   float2 p = __ffma2_rn(f, make_float2(kExp2C3, kExp2C3), make_float2(kExp2C2, kExp2C2));
   p = __ffma2_rn(p, f, make_float2(kExp2C1, kExp2C1));
   p = __ffma2_rn(p, f, make_float2(kExp2C0, kExp2C0));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+  const float2 scale = make_float2(__int_as_float(__float_as_int(t.x) << 23), __int_as_float(__float_as_int(t.y) << 23));
+  return __fmul2_rn(p, scale);
 }
 // 2^x for a pair: on the FMA pipe when `poly`, else two MUFU ex2.approx.
 __device__ __forceinline__ float2 exp2_pair(float2 x, bool poly) {
@@ -302,6 +321,14 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
+}
+
+// Four fp32 values added to global memory at `addr` (16-byte aligned) by the L2's
+// reduction units; no value is returned, so the issuing thread does not wait.
+__device__ __forceinline__ void red_add_f32x4(float* addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(__uint_as_float(a)),
+               "f"(__uint_as_float(b)), "f"(__uint_as_float(c)), "f"(__uint_as_float(d))
+               : "memory");
 }
 
 // Records the first error code in the device status word and raises the CTA's abort flag.

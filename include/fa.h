@@ -63,6 +63,10 @@ typedef enum {
 } fa_status;
 
 /* Forward, bf16 in / bf16 out, fp32 accumulation (tcgen05 tensor cores).
+ * Q/K/V tiles staged on chip and an online softmax with a running max and sum
+ * that rescales the partial output ("LLM paper notes #8: FlashAttention",
+ * adg.csdn.net, sections "tiling" and "online softmax"); lse is saved for the
+ * backward ("recomputation").
  *   q, k, v : (B,H,N,D) bf16, read only.
  *   o       : (B,H,N,D) bf16, written (O = P V, rounded to nearest even).
  *   lse     : (B,H,N) float32, written (natural-log logsumexp of scale*q.k).
@@ -85,27 +89,50 @@ int fa_fwd_f16(const void* q, const void* k, const void* v, void* o, float* lse,
 
 /* Forward in fp32 throughout (fp32 in, fp32 FFMA arithmetic, fp32 out), for
  * callers that need ~1e-6 relative accuracy.  Same arguments as fa_fwd with
- * float32 tensors. */
+ * float32 tensors.  Computes the same tiled online softmax as fa_fwd ("LLM paper
+ * notes #8: FlashAttention", adg.csdn.net, sections "tiling" and "online
+ * softmax"), with every product and exponential in fp32. */
 int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
                int B, int H, int N, int D, float scale, int causal, void* stream);
 
-/* Bytes of device workspace fa_bwd needs.  With Npad = N rounded up to a
- * multiple of 128, the workspace holds two float32 arrays of B*H*Npad rows:
- *   [0, B*H*Npad)            nl_i    = -lse_i * log2(e)   (padding rows: -inf)
- *   [B*H*Npad, 2*B*H*Npad)   delta_i = sum_d dO_id * O_id (padding rows: 0)
- * i.e. 8 * B * H * Npad bytes (a multiple of 1024).  Returns 0 for an
- * unsupported shape. */
+/* ---------------------------------------------------------------------------
+ * Backward.  The gradients of O = softmax(S) V for a scalar loss, with P
+ * recomputed from lse instead of stored ("LLM paper notes #8: FlashAttention",
+ * adg.csdn.net, section "recomputation"; guanweilu.cn, section "three tricks"):
+ *     dV = P^T dO,  dP = dO V^T,  delta_i = sum_d dO_id O_id,
+ *     dS = P * (dP - delta),  dQ = scale dS K,  dK = scale dS^T Q.
+ * Workspace layout (device memory owned by the caller, 16-byte aligned), with
+ * Npad = N rounded up to a multiple of 128 and R = B*H*Npad rows:
+ *   [0, R) floats            nl_i    = -lse_i * log2(e)   (padding rows: -inf)
+ *   [R, 2R) floats           delta_i = sum_d dO_id * O_id (padding rows: 0)
+ *   [2R, 2R + R*DK) floats   fp32 dQ accumulator of fa_bwd (head dims up to 128;
+ *                            DK = 64 for D <= 64, 128 for D in {96, 128}); per
+ *                            128-row query tile a block of 128 x DK floats laid
+ *                            out [DK/4][128 rows][4].
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of device workspace fa_bwd and fa_bwd_f16 need: 4 * R * (2 + DK) for
+ * D <= 128 (statistics and dQ accumulator), 8 * R for D = 256 (statistics only).
+ * A multiple of 1024.  Returns 0 for an unsupported shape. */
 size_t fa_bwd_workspace_size(int B, int H, int N, int D);
+
+/* Bytes of device workspace fa_bwd_deterministic and its stages (fa_bwd_dkdv,
+ * fa_bwd_dq) need: the statistics only, 8 * R.  Returns 0 for an unsupported shape. */
+size_t fa_bwd_deterministic_workspace_size(int B, int H, int N, int D);
 
 /* Backward, bf16 (recomputes P from lse; never stores an N x N matrix).
  *   q, k, v, o, dO : (B,H,N,D) bf16 inputs; o and lse must be the outputs of
  *                    fa_fwd for the same q, k, v, scale and causal.
  *   lse            : (B,H,N) float32 from fa_fwd.
  *   dq, dk, dv     : (B,H,N,D) bf16, overwritten (not accumulated into).
- *   workspace      : device buffer of at least fa_bwd_workspace_size() bytes,
- *                    16-byte aligned; contents on entry ignored, clobbered on exit.
- * Equivalent to fa_bwd_preprocess, then fa_bwd_dkdv and fa_bwd_dq on the
- * same stream. */
+ *   workspace      : device buffer of at least fa_bwd_workspace_size() bytes;
+ *                    contents on entry ignored, clobbered on exit.
+ * For D <= 128 one kernel per 128-key tile computes dK, dV and each tile's
+ * contribution dS K to dQ, which it adds into the workspace's fp32 accumulator
+ * with reductions in L2; equivalent to fa_bwd_preprocess, fa_bwd_dkdvdq and
+ * fa_bwd_dq_finish on the same stream.  The order of those fp32 additions varies
+ * from run to run, so dQ is reproducible to rounding (not bit for bit); dK and
+ * dV are.  For D = 256 it runs the three-stage path of fa_bwd_deterministic. */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dO,
            const float* lse, void* dq, void* dk, void* dv,
            void* workspace, size_t workspace_bytes,
@@ -120,21 +147,49 @@ int fa_bwd_f16(const void* q, const void* k, const void* v, const void* o, const
                void* workspace, size_t workspace_bytes,
                int B, int H, int N, int D, float scale, int causal, void* stream);
 
-/* Backward stage 1: fills the workspace (layout above) from O, dO and lse. */
+/* Backward, bf16 only, bit-for-bit reproducible: the same formulas as fa_bwd in
+ * three stages with no atomics (fa_bwd_preprocess, fa_bwd_dkdv, fa_bwd_dq):
+ * every output tile is owned by one CTA, at the price of a second pass that
+ * recomputes S and dP for dQ.  Workspace: at least
+ * fa_bwd_deterministic_workspace_size() bytes (fa_bwd's workspace also fits). */
+int fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const void* dO,
+                         const float* lse, void* dq, void* dk, void* dv,
+                         void* workspace, size_t workspace_bytes,
+                         int B, int H, int N, int D, float scale, int causal, void* stream);
+
+/* Backward stage 1 (bf16): fills nl and delta from O, dO and lse (delta is the
+ * row sum the softmax gradient subtracts, "recomputation", adg.csdn.net).  When
+ * the workspace holds the dQ accumulator (workspace_bytes >=
+ * fa_bwd_workspace_size and D <= 128) it is zeroed too. */
 int fa_bwd_preprocess(const void* o, const void* dO, const float* lse,
                       void* workspace, size_t workspace_bytes,
                       int B, int H, int N, int D, void* stream);
 
-/* Backward stage 2: dK, dV (bf16, overwritten), reading the workspace that
+/* Fused backward stage 2 (bf16, D <= 128): dK, dV (overwritten) and the dQ
+ * contributions added into the accumulator that fa_bwd_preprocess zeroed.  Each
+ * 128-key tile is owned by one CTA that walks the query tiles, recomputing P
+ * from lse ("recomputation", adg.csdn.net).  Workspace: fa_bwd_workspace_size(). */
+int fa_bwd_dkdvdq(const void* q, const void* k, const void* v, const void* dO,
+                  void* workspace, size_t workspace_bytes, void* dk, void* dv,
+                  int B, int H, int N, int D, float scale, int causal, void* stream);
+
+/* Fused backward stage 3 (bf16, D <= 128): dq = scale * accumulator, rounded to
+ * bf16 (the "dQ finish" of the backward).  Workspace: fa_bwd_workspace_size(). */
+int fa_bwd_dq_finish(const void* workspace, size_t workspace_bytes, void* dq,
+                     int B, int H, int N, int D, float scale, void* stream);
+
+/* Deterministic stage 2 (bf16): dK, dV (overwritten), reading the statistics that
  * stage 1 filled.  Each 128-key tile is owned by one CTA that walks the query
- * rows, so dK and dV need no atomics. */
+ * rows, recomputing P from lse ("recomputation", adg.csdn.net), so dK and dV
+ * need no atomics.  Workspace: fa_bwd_deterministic_workspace_size(). */
 int fa_bwd_dkdv(const void* q, const void* k, const void* v, const void* dO,
                 const void* workspace, size_t workspace_bytes, void* dk, void* dv,
                 int B, int H, int N, int D, float scale, int causal, void* stream);
 
-/* Backward stage 3: dQ (bf16, overwritten), reading the workspace that stage 1
- * filled.  Each 256-query block is owned by one CTA that walks the key tiles,
- * so dQ needs no atomics. */
+/* Deterministic stage 3 (bf16): dQ (overwritten), reading the statistics that
+ * stage 1 filled.  Each 256-query block is owned by one CTA that walks the key
+ * tiles and recomputes S, P and dP for them, so dQ needs no atomics.
+ * Workspace: fa_bwd_deterministic_workspace_size(). */
 int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
               const void* workspace, size_t workspace_bytes, void* dq,
               int B, int H, int N, int D, float scale, int causal, void* stream);
@@ -142,19 +197,21 @@ int fa_bwd_dq(const void* q, const void* k, const void* v, const void* dO,
 /* Size of the fixed device scratch array that fa_bwd_noalloc uses (8 MiB). */
 #define FA_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 
-/* Backward that allocates nothing and takes no workspace.  The paper has no
- * counterpart to this entry point; it exists for callers that cannot allocate
- * device memory -- code that a host framework hands only its input and output
- * buffers, with all device memory planned up front and no workspace or allocator
- * available to the operator.
- *   Same arguments, layout, results and errors as fa_bwd, minus the workspace.
+/* Backward that allocates nothing and takes no workspace (bf16 only).  The paper
+ * has no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory -- code that a host framework hands only its input and
+ * output buffers, with all device memory planned up front and no workspace or
+ * allocator available to the operator.
+ *   Same arguments, layout and errors as fa_bwd_deterministic minus the workspace,
+ *     and the same results bit for bit (it runs the same three kernels).
  *   Scratch: a fixed FA_NOALLOC_SCRATCH_BYTES array in the library's own device
  *     memory (held by every GPU that loads the library until the process exits).
- *     Limit: fa_bwd_workspace_size(B, H, N, D) <= FA_NOALLOC_SCRATCH_BYTES,
+ *     Limit: fa_bwd_deterministic_workspace_size(B, H, N, D) <= FA_NOALLOC_SCRATCH_BYTES,
  *     i.e. B*H*ceil(N/128)*128 <= 1,048,576 rows; larger problems return
  *     FA_ERR_NOALLOC_CAPACITY before anything is launched.
  *   Set-up: the first call on a device looks up the array's device address
  *     (with that device current); make that first call before any stream capture.
+ *     A failed lookup is not remembered: the next call on that device tries again.
  *   Sharing: every call uses the same array; nothing in it needs to start at zero
  *     (each call rewrites what it reads), but calls whose work overlaps on the GPU
  *     (unordered streams) race on it. */

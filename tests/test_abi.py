@@ -30,19 +30,27 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for code in range(11):
+    for code in range(12):
         assert fa.status_string(code).startswith("FA_")
     assert fa.status_string(999) == "unknown fa_status"
 
 
 def test_workspace_size():
-    # two float32 arrays (-lse*log2 e and delta) of B*H*ceil(N/128)*128 rows
-    assert fa.fa_bwd_workspace_size(1, 8, 65536, 128) == 2 * 8 * 65536 * 4
-    assert fa.fa_bwd_workspace_size(1, 1, 3, 64) == 2 * 128 * 4
-    assert fa.fa_bwd_workspace_size(2, 3, 129, 64) == 2 * 6 * 256 * 4
-    assert fa.fa_bwd_workspace_size(1, 1, 128, 96) == 2 * 128 * 4
+    # fa_bwd: two float32 statistics (-lse*log2 e and delta) per padded row, plus the fp32
+    # dQ accumulator of DK floats per padded row (DK = 64 for D <= 64, 128 for D in {96, 128});
+    # rows = B*H*ceil(N/128)*128.  D = 256 has no fused path: statistics only.
+    assert fa.fa_bwd_workspace_size(1, 8, 65536, 128) == 8 * 65536 * (2 + 128) * 4
+    assert fa.fa_bwd_workspace_size(1, 1, 3, 64) == 128 * (2 + 64) * 4
+    assert fa.fa_bwd_workspace_size(2, 3, 129, 64) == 6 * 256 * (2 + 64) * 4
+    assert fa.fa_bwd_workspace_size(1, 1, 128, 32) == 128 * (2 + 64) * 4
+    assert fa.fa_bwd_workspace_size(1, 1, 128, 96) == 128 * (2 + 128) * 4
     assert fa.fa_bwd_workspace_size(1, 1, 128, 80) == 0          # unsupported D
     assert fa.fa_bwd_workspace_size(1, 1, 128, 256) == 2 * 128 * 4
+    for args in ((1, 8, 65536, 128), (2, 3, 129, 64), (1, 1, 128, 256), (1, 1, 1, 96)):
+        B, H, N, D = args
+        assert fa.fa_bwd_deterministic_workspace_size(*args) == 2 * B * H * ((N + 127) // 128 * 128) * 4
+        assert fa.fa_bwd_workspace_size(*args) % 1024 == 0
+    assert fa.fa_bwd_deterministic_workspace_size(1, 1, 128, 80) == 0
 
 
 def test_noalloc_capacity_check_needs_no_gpu():
@@ -88,11 +96,14 @@ def test_bwd_rejects_bad_arguments():
     assert lib.fa_bwd(*args, P, ws, 1, 2, 256, 64, 0.125, 0, None) != 6       # reaches the device check
     assert lib.fa_bwd(*args, Z, ws, 1, 2, 256, 64, 0.125, 0, None) == 8       # no workspace
     assert lib.fa_bwd(*args, P, ws - 1, 1, 2, 256, 64, 0.125, 0, None) == 8   # too small
+    # the deterministic path's smaller workspace does not hold fa_bwd's dQ accumulator
+    wsd = lib.fa_bwd_deterministic_workspace_size(1, 2, 256, 64)
+    assert lib.fa_bwd(*args, P, wsd, 1, 2, 256, 64, 0.125, 0, None) == 8
     assert lib.fa_bwd(*args[:8], U, P, ws, 1, 2, 256, 64, 0.125, 0, None) == 4
     assert lib.fa_bwd(*args[:3], Z, *args[4:], P, ws, 1, 2, 256, 64, 0.125, 0, None) == 1
     assert lib.fa_bwd(*args, P, ws, 1, 2, 256, 80, 0.125, 0, None) == 3
     assert lib.fa_bwd(*args, P, ws, 1, 2, 256, 192, 0.125, 0, None) == 3
-    ws1 = lib.fa_bwd_workspace_size(1, 1, 128, 64)
+    ws1 = lib.fa_bwd_deterministic_workspace_size(1, 1, 128, 64)
     assert ws1 == 2 * 128 * 4
     assert lib.fa_bwd_dq(P, P, P, P, P, ws1, Z, 1, 1, 128, 64, 0.1, 0, None) == 1
     assert lib.fa_bwd_dkdv(P, P, P, P, P, ws1, P, U, 1, 1, 128, 64, 0.1, 0, None) == 4
@@ -100,6 +111,37 @@ def test_bwd_rejects_bad_arguments():
     assert lib.fa_bwd_dq(P, P, P, P, U, ws1, P, 1, 1, 128, 64, 0.1, 0, None) == 4
     assert lib.fa_bwd_preprocess(P, P, Z, P, ws1, 1, 1, 128, 64, None) == 1
     assert lib.fa_bwd_preprocess(P, P, P, Z, ws1, 1, 1, 128, 64, None) == 8
+
+
+def test_deterministic_bwd_rejects_bad_arguments():
+    lib = fa.load_library()
+    wsd = lib.fa_bwd_deterministic_workspace_size(1, 2, 256, 64)
+    args = [P] * 9
+    assert lib.fa_bwd_deterministic(*args, P, wsd, 1, 2, 256, 64, 0.125, 0, None) != 6   # reaches the device
+    assert lib.fa_bwd_deterministic(*args, P, wsd - 1, 1, 2, 256, 64, 0.125, 0, None) == 8
+    assert lib.fa_bwd_deterministic(*args, Z, wsd, 1, 2, 256, 64, 0.125, 0, None) == 8
+    assert lib.fa_bwd_deterministic(*args[:2], Z, *args[3:], P, wsd, 1, 2, 256, 64, 0.125, 0, None) == 1
+    assert lib.fa_bwd_deterministic(*args, U, wsd, 1, 2, 256, 64, 0.125, 0, None) == 4
+    assert lib.fa_bwd_deterministic(*args, P, wsd, 1, 2, 256, 48, 0.125, 0, None) == 3
+    assert lib.fa_bwd_deterministic(*args, P, wsd, 1, 2, 256, 64, float("nan"), 0, None) == 10
+
+
+def test_fused_stages_reject_bad_arguments():
+    lib = fa.load_library()
+    ws = lib.fa_bwd_workspace_size(1, 1, 128, 64)
+    wsd = lib.fa_bwd_deterministic_workspace_size(1, 1, 128, 64)
+    assert lib.fa_bwd_dkdvdq(P, P, P, P, P, ws, Z, P, 1, 1, 128, 64, 0.1, 0, None) == 1
+    assert lib.fa_bwd_dkdvdq(P, P, P, P, P, ws, P, U, 1, 1, 128, 64, 0.1, 0, None) == 4
+    assert lib.fa_bwd_dkdvdq(P, P, P, P, P, wsd, P, P, 1, 1, 128, 64, 0.1, 0, None) == 8   # no accumulator
+    assert lib.fa_bwd_dkdvdq(P, P, P, P, P, ws, P, P, 1, 1, 128, 256, 0.1, 0, None) == 3   # D = 256: no fused path
+    assert lib.fa_bwd_dkdvdq(P, P, P, P, P, ws, P, P, 1, 1, 128, 64, 0.1, 5, None) == 10
+    assert lib.fa_bwd_dq_finish(P, ws, Z, 1, 1, 128, 64, 0.1, None) == 1
+    assert lib.fa_bwd_dq_finish(P, ws, U, 1, 1, 128, 64, 0.1, None) == 4
+    assert lib.fa_bwd_dq_finish(P, wsd, P, 1, 1, 128, 64, 0.1, None) == 8
+    assert lib.fa_bwd_dq_finish(Z, ws, P, 1, 1, 128, 64, 0.1, None) == 8
+    assert lib.fa_bwd_dq_finish(P, ws, P, 1, 1, 128, 256, 0.1, None) == 3
+    assert lib.fa_bwd_dq_finish(P, ws, P, 1, 1, 128, 64, -1.0, None) == 10
+    assert lib.fa_bwd_dq_finish(P, ws, P, 0, 1, 128, 64, 0.1, None) == 2
 
 
 def test_binding_requires_cuda_tensors():

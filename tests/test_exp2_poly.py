@@ -45,6 +45,11 @@ def test_float32_evaluation_error_bound():
     # below the clamp the result is tiny, never negative or garbage
     tiny = g.eval_f32(np.array([-126.0, -300.0, -np.inf]), c)
     assert np.all(tiny > 0) and np.all(tiny < 3e-38)
+    # NaN stays NaN (as through the MUFU ex2), so a NaN score is not silently dropped
+    assert np.isnan(g.eval_f32(np.array([np.nan, -np.nan]), c)).all()
+    # 2^n exactly at the integers where the polynomial is exact to its bound
+    ints = np.arange(-125, 11, dtype=np.float64)
+    assert np.all(np.abs(g.eval_f32(ints, c) / np.exp2(ints) - 1.0) < 7.8e-5)
 
 
 def test_minimax_equioscillates():
