@@ -37,4 +37,6 @@ from ._binding import (  # noqa: F401
     workspace_views,
 )
 
+from .shard import head_ranges, shard_view, sharded_attention, sharded_attention_devices  # noqa: F401,E402
+
 __version__ = "2.0.0"

@@ -21,6 +21,10 @@ CSRC = PKG / "csrc"
 INCLUDE = ROOT / "include"
 BUILD = PKG / "_build"
 LIB = PKG / "libfa.so"
+# Test-only build: every pipeline wait limited to 100 clocks (far less than any tile load
+# takes), so that each kernel runs a wait out and takes its error path.
+TIMEOUT_TEST_LIB = PKG / "libfa_timeout_test.so"
+VARIANTS = {"timeout_test": ["-DFA_WAIT_LIMIT_CYCLES=100"]}
 SOURCES = ["fa_api.cu", "fa_fwd_sm100.cu", "fa_fwd_d256_sm100.cu", "fa_fwd_f32.cu", "fa_bwd_sm100.cu",
            "fa_bwd_d256_sm100.cu", "fa_bwd_fused_sm100.cu", "fa_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -34,19 +38,22 @@ def nvcc() -> str:
 
 
 def _deps():
-    return [CSRC / s for s in SOURCES] + list(CSRC.glob("*.cuh")) + list(CSRC.glob("*.h")) + [INCLUDE / "fa.h"]
+    return ([CSRC / s for s in SOURCES] + list(CSRC.glob("*.cuh")) + list(CSRC.glob("*.h")) + [INCLUDE / "fa.h"]
+            + [pathlib.Path(__file__).resolve()])
 
 
 def up_to_date() -> bool:
-    if not LIB.exists():
+    if not LIB.exists() or not TIMEOUT_TEST_LIB.exists():
         return False
-    t = LIB.stat().st_mtime
+    t = min(LIB.stat().st_mtime, TIMEOUT_TEST_LIB.stat().st_mtime)
     return all(p.stat().st_mtime <= t for p in _deps())
 
 
-def _compile(src: str, verbose: bool, ptxas_v: bool) -> pathlib.Path:
-    obj = BUILD / (pathlib.Path(src).stem + ".o")
-    cmd = [nvcc(), *ARCH, *CFLAGS, "-c", str(CSRC / src), "-o", str(obj)]
+def _compile(src: str, verbose: bool, ptxas_v: bool, variant: str = "") -> pathlib.Path:
+    out = BUILD / variant if variant else BUILD
+    out.mkdir(parents=True, exist_ok=True)
+    obj = out / (pathlib.Path(src).stem + ".o")
+    cmd = [nvcc(), *ARCH, *CFLAGS, *VARIANTS.get(variant, []), "-c", str(CSRC / src), "-o", str(obj)]
     if ptxas_v:
         cmd += ["-Xptxas", "-v"]
     if verbose:
@@ -59,21 +66,28 @@ def _compile(src: str, verbose: bool, ptxas_v: bool) -> pathlib.Path:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> pathlib.Path:
-    """Compiles every CUDA source for sm_100a and links libfa.so next to this file."""
-    if not force and not ptxas_v and up_to_date():
-        return LIB
-    BUILD.mkdir(exist_ok=True)
-    with cf.ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose, ptxas_v), SOURCES))
-    tmp = LIB.with_suffix(".so.tmp")
+def _link(objs, lib: pathlib.Path, verbose: bool) -> None:
+    tmp = lib.with_suffix(".so.tmp")
     cmd = [nvcc(), *ARCH, "-shared", "-o", str(tmp), *map(str, objs), "-cudart", "static"]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> pathlib.Path:
+    """Compiles every CUDA source for sm_100a and links libfa.so next to this file, and the
+    test-only libfa_timeout_test.so (the same sources with short pipeline-wait limits)."""
+    if not force and not ptxas_v and up_to_date():
+        return LIB
+    BUILD.mkdir(exist_ok=True)
+    jobs = [(s, "") for s in SOURCES] + [(s, "timeout_test") for s in SOURCES]
+    with cf.ThreadPoolExecutor(max_workers=min(len(jobs), max(4, os.cpu_count() or 4))) as ex:
+        objs = list(ex.map(lambda j: _compile(j[0], verbose, ptxas_v and not j[1], j[1]), jobs))
+    _link(objs[: len(SOURCES)], LIB, verbose)
+    _link(objs[len(SOURCES):], TIMEOUT_TEST_LIB, verbose)
     return LIB
 
 

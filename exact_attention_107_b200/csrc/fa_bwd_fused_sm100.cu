@@ -275,37 +275,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int sw = r & 7;
     float* dq_head = ws_dq + static_cast<size_t>(bh) * Npad * D;
     uint32_t pk[16];                                     // packed P^T of the current tile
+    // dQ of the previous query tile (this thread: query row r, D/4 columns), held in registers
+    // from its drain out of tensor memory until its 16-byte reductions are issued, a few at a
+    // time, between the next tile's dS^T and P^T arithmetic.  Each SM can send only about
+    // 32 bytes per clock towards L2, so the 64 KB of a tile's dQ take ~2000 clocks to leave:
+    // spread over the tile's work they overlap it, issued in one burst they would stall the
+    // warps for that long.
+    constexpr int kCols = D / 4;
+    constexpr int kReds = kCols / 4;                     // reductions per thread per tile: 8 or 4
+    uint32_t held[kCols];
+    float* held_acc = dq_head + 4 * r;
+    auto red_held = [&](int q) {
+      red_add_f32x4(held_acc + (kReds * g + q) * 512, held[4 * q], held[4 * q + 1], held[4 * q + 2], held[4 * q + 3]);
+    };
 
-    // P^T[r][c] = exp2(s * scale * log2e + nl_c), zero where key > query or key >= N.
-    auto p_tile = [&](int i) -> bool {
+    // P^T[r][c] = exp2(s * scale * log2e + nl_c), zero where key > query or key >= N; with
+    // `reds`, issues the held reductions kReds/2 .. kReds-1 along the way.
+    auto p_tile = [&](int i, bool reds) -> bool {
       const int s = i % L::kStages;
       bool ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarQFull + s), (i / L::kStages) & 1, abort_flag));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS), i & 1, abort_flag));
       if (!ok) return false;
       tc_fence_after();
-      uint32_t sr[32];
-      tmem_ld32(tb + kColS + 32 * g, sr);
-      tmem_ld_wait();
-      reg_fence(sr);
-      const float* st = reinterpret_cast<const float*>(smem + L::kOffStat + s * L::kStatBytes) + 32 * g;
+      const float4* st = reinterpret_cast<const float4*>(smem + L::kOffStat + s * L::kStatBytes) + 8 * g;
       const int qc0 = (it0 + i) * 128 + 32 * g;          // query of this thread's column 0
       const bool edge = tail || (CAUSAL && __any_sync(0xffffffffu, qc0 < key + 32));   // warp-uniform
-      float4 nl4[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) nl4[q] = reinterpret_cast<const float4*>(st)[q];
+      // two halves of 16 columns (one TMEM load each), to keep the held dQ values in registers
       auto p_phase = [&](auto masked) {
 #pragma unroll
-        for (int c2 = 0; c2 < 16; ++c2) {
-          const int c = 2 * c2;
-          const float2 nl = (c2 & 1) ? make_float2(nl4[c2 >> 1].z, nl4[c2 >> 1].w)
-                                     : make_float2(nl4[c2 >> 1].x, nl4[c2 >> 1].y);
-          const float2 sv = make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-          float2 p = exp2_pair(__ffma2_rn(sv, sl2, nl), poly_pair(c2));
-          if (decltype(masked)::value) {
-            if (key_oob || (CAUSAL && key > qc0 + c)) p.x = 0.f;
-            if (key_oob || (CAUSAL && key > qc0 + c + 1)) p.y = 0.f;
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t sr[16];
+          tmem_ld16(tb + kColS + 32 * g + 16 * hf, sr);
+          tmem_ld_wait();
+          reg_fence(sr);
+#pragma unroll
+          for (int c4 = 4 * hf; c4 < 4 * hf + 4; ++c4) {
+            const float4 nl = st[c4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int c2 = 2 * c4 + h, c = 2 * c2, cl = c - 16 * hf;
+              const float2 nlp = h ? make_float2(nl.z, nl.w) : make_float2(nl.x, nl.y);
+              const float2 sv = make_float2(__uint_as_float(sr[cl]), __uint_as_float(sr[cl + 1]));
+              float2 p = exp2_pair(__ffma2_rn(sv, sl2, nlp), poly_pair(c2));
+              if (decltype(masked)::value) {
+                if (key_oob || (CAUSAL && key > qc0 + c)) p.x = 0.f;
+                if (key_oob || (CAUSAL && key > qc0 + c + 1)) p.y = 0.f;
+              }
+              pk[c2] = pack16<F16>(p.x, p.y);
+            }
+            if (reds && kReds == 8 && (c4 & 1)) red_held(4 + (c4 >> 1));         // reductions 4..7
+            if (reds && kReds == 4 && (c4 & 3) == 3) red_held(2 + (c4 >> 2));    // reductions 2, 3
           }
-          pk[c2] = pack16<F16>(p.x, p.y);
         }
       };
       if (edge) p_phase(std::true_type{});
@@ -317,36 +337,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
 
-    // dS^T[r][c] = P^T[r][c] * (dP^T[r][c] - delta_c): packed into tensor memory (for dK) and
-    // into the swizzled shared-memory tile (for dQ).
+    // dS^T[r][c] = P^T[r][c] * (dP^T[r][c] - delta_c), in two halves of 16 columns: packed into
+    // tensor memory (for dK) and into the swizzled shared-memory tile (for dQ).
     auto ds_tile = [&](int i) -> bool {
       const int s = i % L::kStages;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), i & 1, abort_flag))) return false;
       tc_fence_after();
-      uint32_t dp[32];
-      tmem_ld32(tb + kColDP + 32 * g, dp);
-      tmem_ld_wait();
-      reg_fence(dp);
-      const float* st = reinterpret_cast<const float*>(smem + L::kOffStat + s * L::kStatBytes) + 128 + 32 * g;
-      float4 dl4[8];
+      const float4* st = reinterpret_cast<const float4*>(smem + L::kOffStat + s * L::kStatBytes + 512) + 8 * g;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) dl4[q] = reinterpret_cast<const float4*>(st)[q];
-      uint32_t dsk[16];
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t dp[16], dsk[8];
+        tmem_ld16(tb + kColDP + 32 * g + 16 * hf, dp);
+        tmem_ld_wait();
+        reg_fence(dp);
 #pragma unroll
-      for (int c2 = 0; c2 < 16; ++c2) {
-        const int c = 2 * c2;
-        const float2 dl = (c2 & 1) ? make_float2(dl4[c2 >> 1].z, dl4[c2 >> 1].w)
-                                   : make_float2(dl4[c2 >> 1].x, dl4[c2 >> 1].y);
-        const float2 dpv = make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1]));
-        const float2 ds = __fmul2_rn(make_float2(unpack16_lo<F16>(pk[c2]), unpack16_hi<F16>(pk[c2])),
-                                     __ffma2_rn(dl, make_float2(-1.f, -1.f), dpv));
-        dsk[c2] = pack16<F16>(ds.x, ds.y);
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const float4 dl = st[4 * hf + c4];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int c2 = 2 * c4 + h, c = 2 * c2;
+            const float2 dlp = h ? make_float2(dl.z, dl.w) : make_float2(dl.x, dl.y);
+            const float2 dpv = make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1]));
+            const uint32_t pp = pk[8 * hf + c2];
+            const float2 ds = __fmul2_rn(make_float2(unpack16_lo<F16>(pp), unpack16_hi<F16>(pp)),
+                                         __ffma2_rn(dlp, make_float2(-1.f, -1.f), dpv));
+            dsk[c2] = pack16<F16>(ds.x, ds.y);
+          }
+        }
+        // packed columns [8 hf, 8 hf + 8) of this warpgroup's range (already read: half 0 read
+        // columns [0, 16)) and 16-byte chunks 2 hf, 2 hf + 1 of its 64-byte part of row r
+        tmem_st8(tb + kColDP + 32 * g + 8 * hf, dsk);
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          *reinterpret_cast<uint4*>(ds_row + ((((g & 1) * 4 + 2 * hf + q) ^ sw) << 4)) =
+              make_uint4(dsk[4 * q], dsk[4 * q + 1], dsk[4 * q + 2], dsk[4 * q + 3]);
       }
-      tmem_st16(tb + kColDP + 32 * g, dsk);
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(ds_row + ((((g & 1) * 4 + q) ^ sw) << 4)) =
-            make_uint4(dsk[4 * q], dsk[4 * q + 1], dsk[4 * q + 2], dsk[4 * q + 3]);
       fence_async_smem();
       tmem_st_wait();
       tc_fence_before();
@@ -354,34 +379,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
 
-    // dQ_i (this thread: query row r, D/4 columns) added into the accumulator tile of query
-    // tile i, laid out [D/4][128 rows][4 floats] so that a warp's reduction covers 512
-    // contiguous bytes.  The tensor-memory columns are released as soon as they are in
-    // registers, before the reductions are issued: the reductions leave the SM at the
-    // memory system's pace while the next products already run.
+    // dQ_i out of tensor memory into `held`; the columns are released at once (the next dP^T
+    // may overwrite them) and the first half of the reductions into the accumulator tile of
+    // query tile i (laid out [D/4][128 rows][4 floats], so that a warp's reduction covers 512
+    // contiguous bytes) is issued while the MMAs compute dV and that dP^T, which the next
+    // dS^T waits for; the second half goes out during the next P^T.
     auto drain = [&](int i) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::kBarDQFull), i & 1, abort_flag))) return false;
       tc_fence_after();
-      float* acc = dq_head + static_cast<size_t>(it0 + i) * 128 * D + 4 * r;
-      constexpr int kCols = D / 4;                       // columns of dQ this warpgroup drains
-      uint32_t v[kCols];
-      if constexpr (kCols == 32) tmem_ld32(tb + kColDQ + 32 * g, v);
-      else tmem_ld16(tb + kColDQ + 16 * g, v);
+      if constexpr (kCols == 32) tmem_ld32(tb + kColDQ + 32 * g, held);
+      else tmem_ld16(tb + kColDQ + 16 * g, held);
       tmem_ld_wait();
-      reg_fence(v);
+      reg_fence(held);
       tc_fence_before();
       mbar_arrive(bar(L::kBarDQEmpty));
+      held_acc = dq_head + static_cast<size_t>(it0 + i) * 128 * D + 4 * r;
 #pragma unroll
-      for (int q = 0; q < kCols / 4; ++q)
-        red_add_f32x4(acc + (kCols / 4 * g + q) * 512, v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      for (int q = 0; q < kReds / 2; ++q) red_held(q);
       return true;
     };
 
-    bool ok = p_tile(0);
+    bool ok = p_tile(0, false);
     for (int i = 0; ok && i < n; ++i) {
       ok = ds_tile(i);
-      if (ok && i + 1 < n) ok = p_tile(i + 1);
-      if (ok) ok = drain(i);
+      if (ok && i + 1 < n) {
+        ok = p_tile(i + 1, i > 0);                       // + second half of dQ_{i-1}'s reductions
+      } else if (ok && i > 0) {
+#pragma unroll
+        for (int q = kReds / 2; q < kReds; ++q) red_held(q);
+      }
+      if (ok) ok = drain(i);                             // + first half of dQ_i's
+    }
+    if (ok) {
+#pragma unroll
+      for (int q = kReds / 2; q < kReds; ++q) red_held(q);   // the last tile's second half
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarAcc), 0, abort_flag));
     if (!ok) {

@@ -2,9 +2,12 @@
 // kernels use: mbarriers (with bounded waits), TMA tensor copies, and the fifth-
 // generation tensor cores (tcgen05 MMA with accumulators in tensor memory).
 //
-// Every wait here is bounded: a wait that exceeds kWaitLimitCycles (about two
-// seconds) or sees the CTA's abort flag returns false instead of spinning on,
-// so a broken pipeline ends with an error status rather than a hung GPU.
+// Every wait here is bounded: a pipeline wait that exceeds kWaitLimitCycles (about two
+// seconds) or sees the CTA's abort flag returns false instead of spinning on, so a
+// broken pipeline ends with an error status rather than a hung GPU.  The waits with
+// which a failing CTA collects its own copies and MMAs before it exits have their own,
+// fixed limit (kDrainLimitCycles).  A test build of the library shortens the pipeline
+// limit (FA_WAIT_LIMIT_CYCLES) so that every pipeline runs out and takes its error path.
 #pragma once
 
 #include <cstdint>
@@ -12,9 +15,14 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#ifndef FA_WAIT_LIMIT_CYCLES
+#define FA_WAIT_LIMIT_CYCLES 4000000000LL
+#endif
+
 namespace fa {
 
-constexpr long long kWaitLimitCycles = 4000000000LL;
+constexpr long long kWaitLimitCycles = FA_WAIT_LIMIT_CYCLES;
+constexpr long long kDrainLimitCycles = 4000000000LL;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -81,12 +89,13 @@ __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, vo
     if (clock64() - t0 > kWaitLimitCycles) return false;
   }
 }
-// Same, ignoring the abort flag (used to drain a CTA's own in-flight copies on the way out).
+// Same, ignoring the abort flag and with the fixed drain limit (used to collect a CTA's own
+// in-flight copies and MMAs on the way out).
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
   const long long t0 = clock64();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > kWaitLimitCycles) return false;
+    if (clock64() - t0 > kDrainLimitCycles) return false;
   }
 }
 
@@ -211,6 +220,11 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
