@@ -24,7 +24,10 @@ LIB = PKG / "libfa.so"
 # Test-only build: every pipeline wait limited to 100 clocks (far less than any tile load
 # takes), so that each kernel runs a wait out and takes its error path.
 TIMEOUT_TEST_LIB = PKG / "libfa_timeout_test.so"
-VARIANTS = {"timeout_test": ["-DFA_WAIT_LIMIT_CYCLES=100"]}
+# Debug build: device-side bounds checks of computed indices and warp-convergence checks at
+# the warp-collective tensor-memory phases (a failed check records FA_ERR_DEBUG_CHECK).
+DEBUG_LIB = PKG / "libfa_debug.so"
+VARIANTS = {"timeout_test": ["-DFA_WAIT_LIMIT_CYCLES=100"], "debug": ["-DFA_DEBUG_CHECKS"]}
 SOURCES = ["fa_api.cu", "fa_fwd_sm100.cu", "fa_fwd_d256_sm100.cu", "fa_fwd_f32.cu", "fa_bwd_sm100.cu",
            "fa_bwd_d256_sm100.cu", "fa_bwd_fused_sm100.cu", "fa_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -43,9 +46,10 @@ def _deps():
 
 
 def up_to_date() -> bool:
-    if not LIB.exists() or not TIMEOUT_TEST_LIB.exists():
+    libs = (LIB, TIMEOUT_TEST_LIB, DEBUG_LIB)
+    if not all(lib.exists() for lib in libs):
         return False
-    t = min(LIB.stat().st_mtime, TIMEOUT_TEST_LIB.stat().st_mtime)
+    t = min(lib.stat().st_mtime for lib in libs)
     return all(p.stat().st_mtime <= t for p in _deps())
 
 
@@ -78,16 +82,19 @@ def _link(objs, lib: pathlib.Path, verbose: bool) -> None:
 
 
 def build(force: bool = False, verbose: bool = False, ptxas_v: bool = False) -> pathlib.Path:
-    """Compiles every CUDA source for sm_100a and links libfa.so next to this file, and the
-    test-only libfa_timeout_test.so (the same sources with short pipeline-wait limits)."""
+    """Compiles every CUDA source for sm_100a and links libfa.so next to this file, the
+    test-only libfa_timeout_test.so (the same sources with short pipeline-wait limits) and
+    libfa_debug.so (the same sources with device-side bounds and convergence checks)."""
     if not force and not ptxas_v and up_to_date():
         return LIB
     BUILD.mkdir(exist_ok=True)
-    jobs = [(s, "") for s in SOURCES] + [(s, "timeout_test") for s in SOURCES]
+    jobs = [(s, v) for v in ("", "timeout_test", "debug") for s in SOURCES]
     with cf.ThreadPoolExecutor(max_workers=min(len(jobs), max(4, os.cpu_count() or 4))) as ex:
         objs = list(ex.map(lambda j: _compile(j[0], verbose, ptxas_v and not j[1], j[1]), jobs))
-    _link(objs[: len(SOURCES)], LIB, verbose)
-    _link(objs[len(SOURCES):], TIMEOUT_TEST_LIB, verbose)
+    n = len(SOURCES)
+    _link(objs[:n], LIB, verbose)
+    _link(objs[n:2 * n], TIMEOUT_TEST_LIB, verbose)
+    _link(objs[2 * n:], DEBUG_LIB, verbose)
     return LIB
 
 

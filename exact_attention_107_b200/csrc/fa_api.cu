@@ -139,6 +139,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA runtime error";
     case FA_ERR_ARG: return "FA_ERR_ARG: invalid argument";
     case FA_ERR_NOALLOC_CAPACITY: return "FA_ERR_NOALLOC_CAPACITY: problem exceeds the fa_bwd_noalloc scratch size";
+    case FA_ERR_DEBUG_CHECK: return "FA_ERR_DEBUG_CHECK: a device-side check of the debug build failed";
     default: return "unknown fa_status";
   }
 }
@@ -213,7 +214,7 @@ int fa_fwd_f32(const float* q, const float* k, const float* v, float* o, float* 
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
   return launch_status(
-      fa::launch_fwd_f32(q, k, v, o, lse, B * H, N, D, scale, causal, static_cast<cudaStream_t>(stream)));
+      fa::launch_fwd_f32(q, k, v, o, lse, B * H, N, D, scale, causal, ds->status, static_cast<cudaStream_t>(stream)));
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int D) {
@@ -251,6 +252,7 @@ static int preprocess16(const void* o, const void* dO, const float* lse, void* w
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
   a.f16 = f16 ? 1 : 0;
+  a.status = ds->status;
   a.o = o;
   a.dO = dO;
   a.lse = lse;
@@ -341,6 +343,7 @@ static int dq_finish16(const void* workspace, size_t workspace_bytes, void* dq, 
   DeviceState* ds = nullptr;
   if ((st = device_state(&ds)) != FA_OK) return st;
   a.f16 = f16 ? 1 : 0;
+  a.status = ds->status;
   a.BH = B * H;
   a.N = N;
   a.D = D;

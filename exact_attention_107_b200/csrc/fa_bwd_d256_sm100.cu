@@ -139,6 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
+    FA_CONVERGED(status);
     tmem_alloc(smem_u32(slot), 512);
     tmem_relinquish();
   }
@@ -242,11 +243,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q0 = (it0 + i) * 128;
       // this warpgroup's 32 query statistics in the padded workspace (in bounds, 16-byte aligned)
       const size_t srow = static_cast<size_t>(bh) * Npad + q0 + 32 * g;
+      const bool sin = FA_BOUNDS(srow + 32 <= static_cast<size_t>(BH) * Npad, status);
       float4 nl4[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) nl4[q] = __ldg(reinterpret_cast<const float4*>(ws_nl + srow) + q);
+      for (int q = 0; q < 8; ++q)
+        nl4[q] = sin ? __ldg(reinterpret_cast<const float4*>(ws_nl + srow) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS), i & 1, abort_flag));
       if (!ok) break;
+      FA_CONVERGED(status);                                     // warp-collective TMEM loads follow
       tc_fence_after();
       uint32_t sr[32];
       tmem_ld32(tb + kColS + 32 * g, sr);
@@ -279,9 +283,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // dS^T = P^T * (dP^T - delta)
       float4 dl4[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) dl4[q] = __ldg(reinterpret_cast<const float4*>(ws_delta + srow) + q);
+      for (int q = 0; q < 8; ++q)
+        dl4[q] = sin ? __ldg(reinterpret_cast<const float4*>(ws_delta + srow) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), i & 1, abort_flag));
       if (!ok) break;
+      FA_CONVERGED(status);
       tc_fence_after();
       uint32_t dp[32];
       tmem_ld32(tb + kColDP + 32 * g, dp);
@@ -308,6 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       // One 64-column box per warpgroup: dV_h boxes 0-1 (via the idle V tile), dK_h boxes 0-1
       // (via the idle K tile); global columns 128h + 64c.
+      FA_CONVERGED(status);
       tc_fence_after();
       const int wrow = (warp & 3) * 32;
       const bool is_dv = g < 2;
@@ -322,6 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    FA_CONVERGED(status);
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -375,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
+    FA_CONVERGED(status);
     tmem_alloc(smem_u32(slot), 512);
     tmem_relinquish();
   }
@@ -464,8 +473,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tb = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     const int qrow = q0 + r;
     const size_t prow = static_cast<size_t>(bh) * Npad + qrow;         // < B*H*Npad: q0 < N <= Npad
-    const float nl = ws_nl[prow];
-    const float dl = ws_delta[prow];
+    const bool pin = FA_BOUNDS(prow < static_cast<size_t>(BH) * Npad, status);
+    const float nl = pin ? ws_nl[prow] : -CUDART_INF_F;
+    const float dl = pin ? ws_delta[prow] : 0.f;
     const float scale_log2 = scale * kLog2e;
     const float2 sl2 = make_float2(scale_log2, scale_log2), nl2 = make_float2(nl, nl);
     bool ok = true;
@@ -473,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int kc0 = j * 128 + 32 * w;                                 // key of this thread's column 0
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS), j & 1, abort_flag));
       if (!ok) break;
+      FA_CONVERGED(status);                                     // warp-collective TMEM loads follow
       tc_fence_after();
       uint32_t sr[32];
       tmem_ld32(tb + kColS + 32 * w, sr);
@@ -499,6 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       else p_phase(std::false_type{});
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), j & 1, abort_flag));
       if (!ok) break;
+      FA_CONVERGED(status);
       tc_fence_after();
       uint32_t dp[32];
       tmem_ld32(tb + kColDP + 32 * w, dp);
@@ -522,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       raise_error(status, abort_flag, kStatusTimeout);
     } else if (w < 2) {
       // dQ_h box w (64 columns) via the idle Q tile; global columns 128h + 64w
+      FA_CONVERGED(status);
       tc_fence_after();
       stage_box_16<128, F16>(tb + kColDQ, w, scale, smem + L::kOffQ, r);
       store_warp_box_x(&tmdQ, sb + L::kOffQ, w, 2 * h + w, (warp & 3) * 32, q0, bh, lane, N);
@@ -531,6 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    FA_CONVERGED(status);
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

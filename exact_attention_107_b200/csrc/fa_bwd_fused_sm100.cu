@@ -121,6 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
+    FA_CONVERGED(status);
     tmem_alloc(smem_u32(slot), 512);
     tmem_relinquish();
   }
@@ -151,12 +152,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q0 = (it0 + i) * 128;
         if (!(ok = mbar_wait(bar(L::kBarQEmpty + s), ph, abort_flag))) break;
         const uint32_t qf = bar(L::kBarQFull + s);
-        mbar_arrive_expect_tx(qf, T::kBytes + L::kStatBytes);
+        const size_t srow = static_cast<size_t>(bh) * Npad + q0;      // padded rows: always in bounds
+        const bool stats_in = FA_BOUNDS(srow + 128 <= static_cast<size_t>(BH) * Npad, status);
+        mbar_arrive_expect_tx(qf, T::kBytes + (stats_in ? L::kStatBytes : 0));
         for (int c = 0; c < T::kNBox; ++c)
           tma_load_3d(sb + L::kOffQ + s * T::kBytes + c * T::kBox, &tmQ, qf, c * 64, q0, bh);
-        const size_t srow = static_cast<size_t>(bh) * Npad + q0;      // padded rows: always in bounds
-        bulk_load(sb + L::kOffStat + s * L::kStatBytes, ws_nl + srow, 128 * 4, qf);
-        bulk_load(sb + L::kOffStat + s * L::kStatBytes + 128 * 4, ws_delta + srow, 128 * 4, qf);
+        if (stats_in) {
+          bulk_load(sb + L::kOffStat + s * L::kStatBytes, ws_nl + srow, 128 * 4, qf);
+          bulk_load(sb + L::kOffStat + s * L::kStatBytes + 128 * 4, ws_delta + srow, 128 * 4, qf);
+        }
         ++nq;
         if (!(ok = mbar_wait(bar(L::kBarOEmpty + s), ph, abort_flag))) break;
         const uint32_t of = bar(L::kBarOFull + s);
@@ -285,8 +289,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kReds = kCols / 4;                     // reductions per thread per tile: 8 or 4
     uint32_t held[kCols];
     float* held_acc = dq_head + 4 * r;
+    const float* const acc_end = ws_dq + static_cast<size_t>(BH) * Npad * D;   // end of the accumulator
+    (void)acc_end;
     auto red_held = [&](int q) {
-      red_add_f32x4(held_acc + (kReds * g + q) * 512, held[4 * q], held[4 * q + 1], held[4 * q + 2], held[4 * q + 3]);
+      float* a = held_acc + (kReds * g + q) * 512;
+      if (FA_BOUNDS(a >= ws_dq && a + 4 <= acc_end, status)) red_add_f32x4(a, held[4 * q], held[4 * q + 1], held[4 * q + 2], held[4 * q + 3]);
     };
 
     // P^T[r][c] = exp2(s * scale * log2e + nl_c), zero where key > query or key >= N; with
@@ -296,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarQFull + s), (i / L::kStages) & 1, abort_flag));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS), i & 1, abort_flag));
       if (!ok) return false;
+      FA_CONVERGED(status);                              // warp-collective TMEM loads follow
       tc_fence_after();
       const float4* st = reinterpret_cast<const float4*>(smem + L::kOffStat + s * L::kStatBytes) + 8 * g;
       const int qc0 = (it0 + i) * 128 + 32 * g;          // query of this thread's column 0
@@ -342,6 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto ds_tile = [&](int i) -> bool {
       const int s = i % L::kStages;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), i & 1, abort_flag))) return false;
+      FA_CONVERGED(status);
       tc_fence_after();
       const float4* st = reinterpret_cast<const float4*>(smem + L::kOffStat + s * L::kStatBytes + 512) + 8 * g;
 #pragma unroll
@@ -369,6 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st8(tb + kColDP + 32 * g + 8 * hf, dsk);
 #pragma unroll
         for (int q = 0; q < 2; ++q)
+          if (FA_BOUNDS(ds_row + ((((g & 1) * 4 + 2 * hf + q) ^ sw) << 4) + 16 <= smem + L::kOffDS + 2 * L::kDSBox, status))
           *reinterpret_cast<uint4*>(ds_row + ((((g & 1) * 4 + 2 * hf + q) ^ sw) << 4)) =
               make_uint4(dsk[4 * q], dsk[4 * q + 1], dsk[4 * q + 2], dsk[4 * q + 3]);
       }
@@ -386,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dS^T waits for; the second half goes out during the next P^T.
     auto drain = [&](int i) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(bar(L::kBarDQFull), i & 1, abort_flag))) return false;
+      FA_CONVERGED(status);
       tc_fence_after();
       if constexpr (kCols == 32) tmem_ld32(tb + kColDQ + 32 * g, held);
       else tmem_ld16(tb + kColDQ + 16 * g, held);
@@ -420,6 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       // One 64-column box per warpgroup: dV boxes into the V tile, dK boxes into the K tile
       // (the K tile is free: the last dQ product, which reads it, completed before kBarAcc).
+      FA_CONVERGED(status);
       tc_fence_after();
       const int wrow = (warp & 3) * 32;
       const int nbox = T::kNBox;                          // 1 (D=64) or 2 (D=128)
@@ -436,6 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    FA_CONVERGED(status);
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -446,7 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // around in shared memory and written as whole rows of the caller's (B,H,N,D) dQ.
 template <int DK, bool F16>
 __global__ void __launch_bounds__(256) bwd_dq_finish_kernel(const float* __restrict__ acc, uint16_t* __restrict__ dq,
-                                                            int N, int Npad, int D, float scale) {
+                                                            int N, int Npad, int D, float scale, int* status) {
   constexpr int kStride = DK / 4 + 1;                     // float4 per staged row (one of padding)
   __shared__ float4 stage[64 * kStride];
   const long long blk = blockIdx.x;
@@ -457,7 +470,10 @@ __global__ void __launch_bounds__(256) bwd_dq_finish_kernel(const float* __restr
   const float4* src = reinterpret_cast<const float4*>(acc + (bh * Npad + static_cast<long long>(qt) * 128) * DK);
   for (int f = threadIdx.x; f < (DK / 4) * 64; f += 256) {
     const int c4 = f >> 6, rr = f & 63;
-    stage[rr * kStride + c4] = src[c4 * 128 + 64 * h + rr];
+    const float4* sp = src + c4 * 128 + 64 * h + rr;
+    stage[rr * kStride + c4] =
+        FA_BOUNDS(sp + 1 <= reinterpret_cast<const float4*>(acc) + static_cast<long long>(gridDim.x) * 64 * DK / 4, status)
+            ? *sp : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   __syncthreads();
   const int row0 = qt * 128 + 64 * h;
@@ -471,7 +487,9 @@ __global__ void __launch_bounds__(256) bwd_dq_finish_kernel(const float* __restr
     o.y = pack16<F16>(a.z * scale, a.w * scale);
     o.z = pack16<F16>(b.x * scale, b.y * scale);
     o.w = pack16<F16>(b.z * scale, b.w * scale);
-    *reinterpret_cast<uint4*>(dq + (bh * N + row0 + rr) * D + 8 * c8) = o;
+    const long long di = (bh * N + row0 + rr) * D + 8 * c8;
+    if (FA_BOUNDS(di + 8 <= static_cast<long long>(gridDim.x) / (Npad / 64) * N * D, status))
+      *reinterpret_cast<uint4*>(dq + di) = o;
   }
 }
 
@@ -500,7 +518,7 @@ cudaError_t finish_impl(const BwdLaunch& a, void* dq, cudaStream_t stream) {
   const long long blocks = static_cast<long long>(a.BH) * (a.Npad / 64);
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   bwd_dq_finish_kernel<DK, F16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
-      a.ws_dq, static_cast<uint16_t*>(dq), a.N, a.Npad, a.D, a.scale);
+      a.ws_dq, static_cast<uint16_t*>(dq), a.N, a.Npad, a.D, a.scale, a.status);
   return cudaGetLastError();
 }
 

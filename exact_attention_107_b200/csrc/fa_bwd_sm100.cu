@@ -45,7 +45,7 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint16_t* __r
                                                              const float* __restrict__ lse,
                                                              float* __restrict__ ws_nl, float* __restrict__ ws_delta,
                                                              float* __restrict__ ws_dq, int N, int Npad, int D, int DK,
-                                                             long long padded_rows) {
+                                                             long long padded_rows, int* status) {
   const long long gt = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long prow = gt / kLanesPerRow;          // row in the padded (B*H, Npad) layout
   const int part = static_cast<int>(gt % kLanesPerRow);
@@ -54,7 +54,9 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint16_t* __r
   const bool real = prow < padded_rows && n < N;
   const long long row = bh * N + n;                  // row in the caller's (B*H, N) layout
   float acc = 0.f;
-  if (real && part * 8 < D) {
+  const long long rows = padded_rows / Npad * N;       // B*H*N: rows of O, dO and lse
+  (void)rows;
+  if (real && part * 8 < D && FA_BOUNDS(row < rows && (row * D + part * 8 + 8) <= rows * D, status)) {
     const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
     const uint4 b = *reinterpret_cast<const uint4*>(dO + row * D + part * 8);
     const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
@@ -68,12 +70,13 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(const uint16_t* __r
   for (int off = kLanesPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (prow < padded_rows && part == 0) {
     ws_delta[prow] = acc;
-    ws_nl[prow] = real ? -lse[row] * kLog2e : -CUDART_INF_F;
+    ws_nl[prow] = (real && FA_BOUNDS(row < rows, status)) ? -lse[row] * kLog2e : -CUDART_INF_F;
   }
   // The fused backward adds dQ into an fp32 accumulator of DK floats per padded row: zero
   // this row's share of it (the accumulator's tile layout keeps a row's DK floats
   // contiguous only per tile, but zeroing [prow * DK, prow * DK + DK) over all rows covers it).
-  if (ws_dq != nullptr && prow < padded_rows) {
+  if (ws_dq != nullptr && prow < padded_rows &&
+      FA_BOUNDS(prow * DK + (part + 1) * (DK / kLanesPerRow) <= padded_rows * DK, status)) {
     const int per_lane = DK / kLanesPerRow;             // 8 or 16 floats
     float4* z = reinterpret_cast<float4*>(ws_dq + prow * DK + part * per_lane);
     for (int i = 0; i < per_lane / 4; ++i) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -166,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
+    FA_CONVERGED(status);
     tmem_alloc(smem_u32(slot), 512);
     tmem_relinquish();
   }
@@ -197,12 +201,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q0 = (it0 + i) * 128;
         if (!(ok = mbar_wait(bar(L::kBarQEmpty + s), ph, abort_flag))) break;
         const uint32_t qf = bar(L::kBarQFull + s);
-        mbar_arrive_expect_tx(qf, T::kBytes + L::kStatBytes);
+        const size_t srow = static_cast<size_t>(bh) * Npad + q0;      // padded rows: always in bounds
+        const bool stats_in = FA_BOUNDS(srow + 128 <= static_cast<size_t>(BH) * Npad, status);
+        mbar_arrive_expect_tx(qf, T::kBytes + (stats_in ? L::kStatBytes : 0));
         for (int c = 0; c < T::kNBox; ++c)
           tma_load_3d(sb + L::kOffQ + s * T::kBytes + c * T::kBox, &tmQ, qf, c * 64, q0, bh);
-        const size_t srow = static_cast<size_t>(bh) * Npad + q0;      // padded rows: always in bounds
-        bulk_load(sb + L::kOffStat + s * L::kStatBytes, ws_nl + srow, 128 * 4, qf);
-        bulk_load(sb + L::kOffStat + s * L::kStatBytes + 128 * 4, ws_delta + srow, 128 * 4, qf);
+        if (stats_in) {
+          bulk_load(sb + L::kOffStat + s * L::kStatBytes, ws_nl + srow, 128 * 4, qf);
+          bulk_load(sb + L::kOffStat + s * L::kStatBytes + 128 * 4, ws_delta + srow, 128 * 4, qf);
+        }
         ++nq;
         if (!(ok = mbar_wait(bar(L::kBarOEmpty + s), ph, abort_flag))) break;
         const uint32_t of = bar(L::kBarOFull + s);
@@ -299,6 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarQFull + s), (i / L::kStages) & 1, abort_flag));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS), i & 1, abort_flag));
       if (!ok) break;
+      FA_CONVERGED(status);                                     // warp-collective TMEM loads follow
       tc_fence_after();
       uint32_t sr[32];
       tmem_ld32(tb + kColS + 32 * g, sr);
@@ -338,6 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // dS^T[r][c] = P^T[r][c] * (dP^T[r][c] - delta_c)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP), i & 1, abort_flag));
       if (!ok) break;
+      FA_CONVERGED(status);
       tc_fence_after();
       uint32_t dp[32];
       tmem_ld32(tb + kColDP + 32 * g, dp);
@@ -366,6 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       raise_error(status, abort_flag, kStatusTimeout);
     } else {
       // One 64-column box per warpgroup: dV boxes into the V tile, dK boxes into the K tile.
+      FA_CONVERGED(status);
       tc_fence_after();
       const int wrow = (warp & 3) * 32;
       const int nbox = T::kNBox;                                         // 1 (D=64) or 2 (D=128)
@@ -382,6 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    FA_CONVERGED(status);
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -471,6 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
+    FA_CONVERGED(status);
     tmem_alloc(smem_u32(slot), 512);
     tmem_relinquish();
   }
@@ -602,13 +614,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     if (nk[t] > 0) {
       const size_t prow = static_cast<size_t>(bh) * Npad + qrow;       // < B*H*Npad: q0[t] < N <= Npad
-      const float nl = ws_nl[prow];
-      const float dl = ws_delta[prow];
+      const bool in = FA_BOUNDS(prow < static_cast<size_t>(BH) * Npad, status);
+      const float nl = in ? ws_nl[prow] : -CUDART_INF_F;
+      const float dl = in ? ws_delta[prow] : 0.f;
       const float scale_log2 = scale * kLog2e;
       for (int j = 0; j < nk[t]; ++j) {
         const int kv0 = j * 128 + 64 * h;                               // key of this thread's column 0
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarS + t), j & 1, abort_flag));
         if (!ok) break;
+        FA_CONVERGED(status);                                   // warp-collective TMEM loads follow
         tc_fence_after();
         // keep key columns c <= lim (causal diagonal, keys past N)
         const int lim = min(CAUSAL ? qrow - kv0 : 63, N - 1 - kv0);
@@ -644,6 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(L::kBarSC + t));                   // S_t has been read: dP_t may overwrite it
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarDP + t), j & 1, abort_flag));
         if (!ok) break;
+        FA_CONVERGED(status);
         tc_fence_after();
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
@@ -672,6 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         raise_error(status, abort_flag, kStatusTimeout);
       } else if (h < T::kNBox) {
         // dQ_t box h (64 columns) into the idle Q_t tile, then TMA
+        FA_CONVERGED(status);
         tc_fence_after();
         stage_box_16<D, F16>(tb + 256 + D * t, h, scale, smem + L::kOffQ + t * T::kBytes, r);
         store_warp_box<D>(&tmdQ, sb + L::kOffQ + t * T::kBytes, h, (warp & 3) * 32, q0[t], bh, lane, N);
@@ -682,6 +698,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    FA_CONVERGED(status);
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -695,7 +712,7 @@ cudaError_t preprocess_impl(const BwdLaunch& a, cudaStream_t stream) {
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   bwd_preprocess_kernel<kLanesPerRow, F16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
       static_cast<const uint16_t*>(a.o), static_cast<const uint16_t*>(a.dO), a.lse, a.ws_nl, a.ws_delta,
-      a.ws_dq, a.N, a.Npad, a.D, a.DK, padded_rows);
+      a.ws_dq, a.N, a.Npad, a.D, a.DK, padded_rows, a.status);
   return cudaGetLastError();
 }
 

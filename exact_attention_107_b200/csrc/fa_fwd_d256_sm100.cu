@@ -107,6 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
+    FA_CONVERGED(status);
     tmem_alloc(smem_u32(slot), 512);
     tmem_relinquish();
   }
@@ -213,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tS = tmem + lane_off + (j & 1) * 128;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarSFull + (j & 1)), (j >> 1) & 1, abort_flag));
       if (!ok) break;
+      FA_CONVERGED(status);                                     // warp-collective TMEM loads follow
       tc_fence_after();
       uint32_t sr[4][32];
       tmem_ld32(tS, sr[0]);
@@ -263,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ODone).  PV_j cannot start before this thread arrives on PFull below.
         ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarODone), (j - 1) & 1, abort_flag));
         if (!ok) break;
+        FA_CONVERGED(status);
         tc_fence_after();
 #pragma unroll
         for (int cc = 0; cc < kD / 32; ++cc) {
@@ -288,6 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok) {
       raise_error(status, abort_flag, kStatusTimeout);
     } else {
+      FA_CONVERGED(status);
       tc_fence_after();
       // Epilogue: O / l -> 16-bit into this warp's 32 rows of the (now idle) Q tile, in
       // the 128-byte-swizzled layout of the O tensor map, then one TMA store per box.
@@ -320,13 +324,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_commit();
         bulk_wait_read0();
       }
-      if (qrow < N) lse[static_cast<size_t>(bh) * N + qrow] = m * kLn2 + logf(l);
+      if (qrow < N && FA_BOUNDS(static_cast<size_t>(bh) < static_cast<size_t>(BH), status))
+        lse[static_cast<size_t>(bh) * N + qrow] = m * kLn2 + logf(l);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    FA_CONVERGED(status);
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

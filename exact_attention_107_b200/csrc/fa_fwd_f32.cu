@@ -13,6 +13,7 @@
 #include <math_constants.h>
 
 #include "fa_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace fa {
 namespace {
@@ -33,7 +34,7 @@ struct F32Smem {
 template <int D>
 __global__ void __launch_bounds__(kThreads)
     fwd_f32_kernel(const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
-                   float* __restrict__ o, float* __restrict__ lse, int N, float scale, int causal) {
+                   float* __restrict__ o, float* __restrict__ lse, int N, float scale, int causal, int* status) {
   using L = F32Smem<D>;
   extern __shared__ float sm[];
   float* sQ = sm;
@@ -44,10 +45,14 @@ __global__ void __launch_bounds__(kThreads)
   const int tid = threadIdx.x, ty = tid >> 3, tx = tid & 7;
   const int q0 = blockIdx.x * kBM;
   const size_t base = static_cast<size_t>(blockIdx.y) * N * D;
+  const size_t total = static_cast<size_t>(gridDim.y) * N * D;   // elements of each (B,H,N,D) tensor
+  (void)total;
+  (void)status;
 
   for (int i = tid; i < kBM * D; i += kThreads) {
     const int r = i / D, d = i % D;
-    sQ[r * L::kQStride + d] = (q0 + r < N) ? q[base + static_cast<size_t>(q0 + r) * D + d] : 0.f;
+    const size_t gi = base + static_cast<size_t>(q0 + r) * D + d;
+    sQ[r * L::kQStride + d] = (q0 + r < N && FA_BOUNDS(gi < total, status)) ? q[gi] : 0.f;
   }
 
   float acc[2][D / 8];
@@ -66,9 +71,10 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();   // previous tile's sK / sV / sP no longer in use
     for (int i = tid; i < kBN * D; i += kThreads) {
       const int r = i / D, d = i % D;
-      const bool in = kv0 + r < N;
-      sK[r * L::kKStride + d] = in ? k[base + static_cast<size_t>(kv0 + r) * D + d] : 0.f;
-      sV[r * D + d] = in ? v[base + static_cast<size_t>(kv0 + r) * D + d] : 0.f;
+      const size_t gi = base + static_cast<size_t>(kv0 + r) * D + d;
+      const bool in = kv0 + r < N && FA_BOUNDS(gi < total, status);
+      sK[r * L::kKStride + d] = in ? k[gi] : 0.f;
+      sV[r * D + d] = in ? v[gi] : 0.f;
     }
     __syncthreads();
     float s[2][4];
@@ -136,30 +142,34 @@ __global__ void __launch_bounds__(kThreads)
     if (rows[i] >= N) continue;
     const float inv = 1.f / l[i];
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) o[base + static_cast<size_t>(rows[i]) * D + tx + 8 * c] = acc[i][c] * inv;
-    if (tx == 0) lse[static_cast<size_t>(blockIdx.y) * N + rows[i]] = m[i] + logf(l[i]);
+    for (int c = 0; c < D / 8; ++c) {
+      const size_t gi = base + static_cast<size_t>(rows[i]) * D + tx + 8 * c;
+      if (FA_BOUNDS(gi < total, status)) o[gi] = acc[i][c] * inv;
+    }
+    const size_t li = static_cast<size_t>(blockIdx.y) * N + rows[i];
+    if (tx == 0 && FA_BOUNDS(li < static_cast<size_t>(gridDim.y) * N, status)) lse[li] = m[i] + logf(l[i]);
   }
 }
 
 template <int D>
 cudaError_t launch_impl(const float* q, const float* k, const float* v, float* o, float* lse, int BH, int N,
-                        float scale, int causal, cudaStream_t stream) {
+                        float scale, int causal, int* status, cudaStream_t stream) {
   using L = F32Smem<D>;
   cudaError_t e = cudaFuncSetAttribute(fwd_f32_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
   if (e != cudaSuccess) return e;
   const dim3 grid((N + kBM - 1) / kBM, BH);
-  fwd_f32_kernel<D><<<grid, kThreads, L::kBytes, stream>>>(q, k, v, o, lse, N, scale, causal);
+  fwd_f32_kernel<D><<<grid, kThreads, L::kBytes, stream>>>(q, k, v, o, lse, N, scale, causal, status);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int BH, int N,
-                           int D, float scale, int causal, cudaStream_t stream) {
+                           int D, float scale, int causal, int* status, cudaStream_t stream) {
   switch (D) {
-    case 32: return launch_impl<32>(q, k, v, o, lse, BH, N, scale, causal, stream);
-    case 64: return launch_impl<64>(q, k, v, o, lse, BH, N, scale, causal, stream);
-    default: return launch_impl<128>(q, k, v, o, lse, BH, N, scale, causal, stream);
+    case 32: return launch_impl<32>(q, k, v, o, lse, BH, N, scale, causal, status, stream);
+    case 64: return launch_impl<64>(q, k, v, o, lse, BH, N, scale, causal, status, stream);
+    default: return launch_impl<128>(q, k, v, o, lse, BH, N, scale, causal, status, stream);
   }
 }
 

@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
+    FA_CONVERGED(status);
     tmem_alloc(smem_u32(slot), 512);
     tmem_relinquish();
   }
@@ -260,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < nkv[t]; ++j) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(L::kBarSFull + t), j & 1, abort_flag));
       if (!ok) break;
+      FA_CONVERGED(status);                                     // warp-collective TMEM loads follow
       tc_fence_after();
       uint32_t sr[4][32];
       tmem_ld32(tS, sr[0]);
@@ -309,6 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[c2] = pack16<F16>(p.x, p.y);
         }
         if (h == 0 && j > 0 && __any_sync(0xffffffffu, need)) {
+          FA_CONVERGED(status);
           // Rescale O_t before any of this step's P V products lands in it (after the
           // first half's exponentials, whose scores no longer occupy registers).  O_t was
           // finished by the PV MMAs of step j-1: the commit that announced S_t(j) also
@@ -341,6 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok) {
       raise_error(status, abort_flag, kStatusTimeout);
     } else if (nkv[t] > 0) {
+      FA_CONVERGED(status);
       tc_fence_after();
       // Epilogue: O / l -> bf16 / fp16 into this warp's 32 rows of the (now idle) Q_t tile,
       // in the 128-byte-swizzled layout the O tensor map expects, then one TMA store
@@ -374,13 +378,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_commit();
         bulk_wait_read0();
       }
-      if (qrow < N) lse[static_cast<size_t>(bh) * N + qrow] = m * kLn2 + logf(l);
+      if (qrow < N && FA_BOUNDS(static_cast<size_t>(bh) < static_cast<size_t>(BH), status))
+        lse[static_cast<size_t>(bh) * N + qrow] = m * kLn2 + logf(l);
     }
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    FA_CONVERGED(status);
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

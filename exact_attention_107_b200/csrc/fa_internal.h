@@ -44,7 +44,7 @@ cudaError_t launch_fwd_d256(const FwdLaunch& a, cudaStream_t stream);
 
 // fp32 forward (fa_fwd_f32.cu), plain pointers.
 cudaError_t launch_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse,
-                           int BH, int N, int D, float scale, int causal, cudaStream_t stream);
+                           int BH, int N, int D, float scale, int causal, int* status, cudaStream_t stream);
 
 // Backward stages (fa_bwd_sm100.cu).  The workspace holds, per (b, h) and per row of
 // N padded up to a multiple of 128 (Npad): ws_nl = -lse * log2(e) (padding: -inf)

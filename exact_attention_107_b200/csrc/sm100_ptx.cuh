@@ -345,6 +345,25 @@ __device__ __forceinline__ void red_add_f32x4(float* addr, uint32_t a, uint32_t 
                : "memory");
 }
 
+// Debug build (compiled with FA_DEBUG_CHECKS): device-side checks of every computed
+// global-memory index and shared-memory offset against its buffer, and of warp convergence
+// at the entry of each phase that issues warp-collective (.sync.aligned) tensor-memory
+// operations.  A failed check records FA_ERR_DEBUG_CHECK in the status word and skips the
+// guarded access, so a wrong index never touches memory outside its buffer.  In the normal
+// build both macros compile to nothing.
+constexpr int kStatusDebugCheck = 12;   // FA_ERR_DEBUG_CHECK
+__device__ __forceinline__ bool debug_check(bool ok, int* status) {
+  if (!ok && status != nullptr) atomicCAS(status, 0, kStatusDebugCheck);
+  return ok;
+}
+#ifdef FA_DEBUG_CHECKS
+#define FA_BOUNDS(cond, status) (::fa::debug_check(static_cast<bool>(cond), (status)))
+#define FA_CONVERGED(status) ((void)::fa::debug_check(__activemask() == 0xffffffffu, (status)))
+#else
+#define FA_BOUNDS(cond, status) true
+#define FA_CONVERGED(status) ((void)0)
+#endif
+
 // Records the first error code in the device status word and raises the CTA's abort flag.
 __device__ __forceinline__ void raise_error(int* status, volatile int* abort_flag, int code) {
   *abort_flag = 1;

@@ -59,7 +59,8 @@ typedef enum {
   FA_ERR_WORKSPACE = 8,        /* workspace NULL or smaller than required         */
   FA_ERR_CUDA = 9,             /* another CUDA runtime error                      */
   FA_ERR_ARG = 10,             /* another invalid argument (scale not finite ...) */
-  FA_ERR_NOALLOC_CAPACITY = 11 /* problem too large for fa_bwd_noalloc's scratch   */
+  FA_ERR_NOALLOC_CAPACITY = 11, /* problem too large for fa_bwd_noalloc's scratch  */
+  FA_ERR_DEBUG_CHECK = 12      /* a device-side check of the debug build failed   */
 } fa_status;
 
 /* Forward, bf16 in / bf16 out, fp32 accumulation (tcgen05 tensor cores).
@@ -224,7 +225,12 @@ const char* fa_status_string(int status);
 
 /* Reads the device status word of the current device (synchronises the
  * device first).  Returns FA_OK or the first FA_ERR_* a kernel recorded;
- * if reset != 0 the word is cleared afterwards. */
+ * if reset != 0 the word is cleared afterwards.  Kernels record
+ * FA_ERR_TIMEOUT (a pipeline wait ran out) and FA_ERR_LAUNCH (a launch they
+ * cannot use); the debug build of the library (libfa_debug.so, compiled with
+ * FA_DEBUG_CHECKS) also records FA_ERR_DEBUG_CHECK when a computed index falls
+ * outside its buffer or a warp reaches a warp-collective tensor-memory
+ * operation diverged, and skips that access instead of performing it. */
 int fa_device_status(int reset);
 
 /* Library version, major*10000 + minor*100 + patch. */

@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for code in range(12):
+    for code in range(13):
         assert fa.status_string(code).startswith("FA_")
     assert fa.status_string(999) == "unknown fa_status"
 
