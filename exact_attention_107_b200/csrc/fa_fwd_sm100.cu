@@ -300,15 +300,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 sl2 = make_float2(scale_log2, scale_log2), neg2 = make_float2(neg, neg);
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
+        // P of keys [64h, 64h+64) as packed pairs, stored 16 pairs at a time (nothing reads
+        // them before this half's barrier arrival below), to keep the registers for S.
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) {
-          const int c = 32 * h + c2;                       // pair index: columns 2c, 2c + 1
-          const float2 sv = make_float2(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]),
-                                        __uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]));
-          const float2 p = exp2_pair(__ffma2_rn(sv, sl2, neg2), poly_pair<D>(c));
-          sum[c & 1] = __fadd2_rn(sum[c & 1], p);
-          pk[c2] = pack16<F16>(p.x, p.y);
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c2 = 0; c2 < 16; ++c2) {
+            const int c = 32 * h + 16 * hh + c2;           // pair index: columns 2c, 2c + 1
+            const float2 sv = make_float2(__uint_as_float(sr[(2 * c) >> 5][(2 * c) & 31]),
+                                          __uint_as_float(sr[(2 * c + 1) >> 5][(2 * c + 1) & 31]));
+            const float2 p = exp2_pair(__ffma2_rn(sv, sl2, neg2), poly_pair<D>(c));
+            sum[c & 1] = __fadd2_rn(sum[c & 1], p);
+            pk[c2] = pack16<F16>(p.x, p.y);
+          }
+          tmem_st16(tS + 32 * h + 16 * hh, pk);
         }
         if (h == 0 && j > 0 && __any_sync(0xffffffffu, need)) {
           FA_CONVERGED(status);
@@ -332,7 +338,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(tO + cc * 32, o);
           }
         }
-        tmem_st32(tS + 32 * h, pk);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar(L::kBarPFull + 2 * h + t));
