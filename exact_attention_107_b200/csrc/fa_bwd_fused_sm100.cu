@@ -186,29 +186,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto sQ = [&](int i) { return sb + L::kOffQ + (i % L::kStages) * T::kBytes; };
       auto sdO = [&](int i) { return sb + L::kOffdO + (i % L::kStages) * T::kBytes; };
       auto phase = [&](int i) { return static_cast<uint32_t>((i / L::kStages) & 1); };
+      // K-major operands: four K-steps of 16 per 64-column box, 32 bytes apart.  MN-major
+      // operands: one K-step per 16 rows (2048 bytes).  Packed 16-bit A operands in tensor
+      // memory: K-steps at columns +0, +8, +32, +40 (see packed_col), then the next 64.
       auto issue_st = [&](int i) {      // S^T = K_j Q_i^T
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + kColS, kmajor_desc(sK, kk, T::kBox), kmajor_desc(sQ(i), kk, T::kBox), kIdS, kk > 0);
+        for (int c = 0; c < D / 64; ++c)
+          mma_ss_x4<2, 4, 6, 2, 4, 6>(tmem + kColS, sdesc_sw128(sK + c * T::kBox, 16, 1024),
+                                      sdesc_sw128(sQ(i) + c * T::kBox, 16, 1024), kIdS, c > 0 ? 1u : 0u);
         tc_commit(bar(L::kBarS));
       };
       auto issue_dpt = [&](int i) {     // dP^T = V_j dO_i^T
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + kColDP, kmajor_desc(sV, kk, T::kBox), kmajor_desc(sdO(i), kk, T::kBox), kIdS, kk > 0);
+        for (int c = 0; c < D / 64; ++c)
+          mma_ss_x4<2, 4, 6, 2, 4, 6>(tmem + kColDP, sdesc_sw128(sV + c * T::kBox, 16, 1024),
+                                      sdesc_sw128(sdO(i) + c * T::kBox, 16, 1024), kIdS, c > 0 ? 1u : 0u);
         tc_commit(bar(L::kBarDP));
       };
       // acc (+)= A_tmem (packed 16-bit, 128 queries) * B_smem (128 queries x D, MN-major)
       auto issue_acc = [&](uint32_t dcol, uint32_t abase, uint32_t b_tile, bool first) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + dcol, tmem + packed_col(abase, kk), mnmajor_desc(b_tile, kk, T::kBox), kIdAcc,
-                 (!first || kk > 0) ? 1u : 0u);
+        for (int g = 0; g < 2; ++g)
+          mma_ts_x4<8, 32, 40, 128, 256, 384>(tmem + dcol, tmem + packed_col(abase, 4 * g),
+                                              sdesc_sw128(b_tile + g * 4 * 2048, T::kBox, 1024), kIdAcc,
+                                              (!first || g > 0) ? 1u : 0u);
       };
       auto issue_dq = [&]() {           // dQ_i = dS_i K_j: 128 queries x D over the 128 keys
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ss(tmem + kColDQ, mnmajor_desc(sDS, kk, L::kDSBox), mnmajor_desc(sK, kk, T::kBox), kIdDQ, kk > 0);
+        for (int g = 0; g < 2; ++g)
+          mma_ss_x4<128, 256, 384, 128, 256, 384>(tmem + kColDQ, sdesc_sw128(sDS + g * 4 * 2048, L::kDSBox, 1024),
+                                                  sdesc_sw128(sK + g * 4 * 2048, T::kBox, 1024), kIdDQ,
+                                                  g > 0 ? 1u : 0u);
         tc_commit(bar(L::kBarDQFull));
       };
       bool ok = mbar_wait_spin(bar(L::kBarKV), 0, abort_flag) &&

@@ -182,24 +182,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_16(kBM, kBN, false, false, F16);  // Q, K both K-major
       constexpr uint32_t kIdO = idesc_16(kBM, D, false, true, F16);    // P from TMEM, V MN-major
+      // Each 64-column box of Q_t and K_j holds four K-steps of 16 (32 bytes apart).
       auto issue_s = [&](int t, int j) {
         const uint32_t qa = sb + L::kOffQ + t * L::kTile;
         const uint32_t kb = sb + L::kOffK + (j % L::kStages) * L::kTile;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kBox + (kk & 3) * 32;
-          mma_ss(tmem + t * 128, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdS,
-                 kk > 0 ? 1u : 0u);
-        }
+        for (int c = 0; c < L::kNBox; ++c)
+          mma_ss_x4<2, 4, 6, 2, 4, 6>(tmem + t * 128, sdesc_sw128(qa + c * L::kBox, 16, 1024),
+                                      sdesc_sw128(kb + c * L::kBox, 16, 1024), kIdS, c > 0 ? 1u : 0u);
         tc_commit(bar(L::kBarSFull + t));
       };
-      // O_t += P_t V_j over keys [64h, 64h+64): K-steps 4h .. 4h+3.
+      // O_t += P_t V_j over keys [64h, 64h+64): K-steps 4h .. 4h+3, each 8 packed P columns
+      // and 16 V rows (2048 bytes) further on.
       auto issue_pv = [&](int t, int j, int h) {
         const uint32_t vb = sb + L::kOffV + (j % L::kStages) * L::kTile;
-#pragma unroll
-        for (int kk = 4 * h; kk < 4 * h + 4; ++kk)
-          mma_ts(tmem + 256 + t * D, tmem + t * 128 + kk * 8, sdesc_sw128(vb + kk * 2048, L::kBox, 1024), kIdO,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+        mma_ts_x4<8, 16, 24, 128, 256, 384>(tmem + 256 + t * D, tmem + t * 128 + 32 * h,
+                                            sdesc_sw128(vb + h * 4 * 2048, L::kBox, 1024), kIdO,
+                                            (j > 0 || h > 0) ? 1u : 0u);
       };
       bool ok = mbar_wait_spin(bar(L::kBarQFull), 0, abort_flag);
       if (ok && nkv_max > 0) {

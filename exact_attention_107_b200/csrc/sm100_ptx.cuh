@@ -82,6 +82,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // thread, which should react to a completed phase at once (the many softmax warps use
 // mbar_wait, whose suspension keeps their polling off the shared-memory pipe).
 __device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_test_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (;;) {
     if (mbar_test_wait(bar, parity)) return true;
@@ -177,6 +178,51 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Four K-steps of one product, issued back to back from precomputed descriptors: step k
+// (k = 0..3) uses the A and B descriptors advanced by the k-th offsets (step 0: none), in
+// the descriptors' 16-byte start-address units.  The sums stay inside the 14-bit
+// start-address field since every shared-memory address here is below 256 KB.  Only
+// step 0 honours `accumulate`; steps 1..3 always accumulate.  The MMA-issuing thread
+// shares its SMSP with busy element-wise warps, so every instruction it saves per MMA
+// shortens the gaps in which the tensor pipe waits for work.
+template <int A1, int A2, int A3, int B1, int B2, int B3>
+__device__ __forceinline__ void mma_ss_x4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t.reg .b64 a, b;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 q, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "add.s64 a, %1, %6;\n\tadd.s64 b, %2, %9;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+      "add.s64 a, %1, %7;\n\tadd.s64 b, %2, %10;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t"
+      "add.s64 a, %1, %8;\n\tadd.s64 b, %2, %11;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, q;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(1u), "n"(A1), "n"(A2), "n"(A3), "n"(B1), "n"(B2),
+      "n"(B3)
+      : "memory");
+}
+// Same with A read from tensor memory: the A offsets are tensor-memory columns.
+template <int A1, int A2, int A3, int B1, int B2, int B3>
+__device__ __forceinline__ void mma_ts_x4(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t.reg .b32 a;\n\t.reg .b64 b;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.ne.b32 q, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.s32 a, %1, %6;\n\tadd.s64 b, %2, %9;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t"
+      "add.s32 a, %1, %7;\n\tadd.s64 b, %2, %10;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t"
+      "add.s32 a, %1, %8;\n\tadd.s64 b, %2, %11;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, q;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(1u), "n"(A1), "n"(A2), "n"(A3), "n"(B1), "n"(B2),
+      "n"(B3)
       : "memory");
 }
 
