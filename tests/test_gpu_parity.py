@@ -272,7 +272,10 @@ def test_c1_fp32_forward():
 
 
 def test_fp32_path_small_shapes():
-    for (B, H, N, D, causal) in [(1, 1, 1, 32, False), (2, 2, 100, 128, True), (1, 3, 333, 64, True)]:
+    # one row, ragged tails, several key chunks of each head dim (chunks of 64 keys at D <= 64
+    # and 32 at D = 128; 8 query rows per CTA)
+    for (B, H, N, D, causal) in [(1, 1, 1, 32, False), (2, 2, 100, 128, True), (1, 3, 333, 64, True),
+                                 (1, 2, 1000, 64, False), (1, 1, 520, 128, True), (2, 1, 97, 32, False)]:
         w = workloads.custom("f32", B, H, N, D, causal, dtype="fp32", seed=3)
         q, k, v, _ = workloads.make_inputs(w, with_grad_out=False)
         O, lse, _ = gpu_forward(q, k, v, w.softmax_scale, causal)
